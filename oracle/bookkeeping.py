@@ -1,0 +1,172 @@
+"""Naive model of PagedAttention's block bookkeeping -- oracle side.
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, the smoke check and the bench's
+CPU-baseline leg, never by the library.  It shares no code with the library's
+C++ block manager; the tests compare the two bit for bit.
+
+What the pages fix, and where:
+
+* the cache is cut into fixed-size blocks, each holding the keys and values of
+  ``block_size`` tokens; a per-sequence block table maps logical block i to a
+  physical block id ("PagedAttention" ops page, Concept -- What it is; "Paged
+  Attention" KV-cache lesson, analogy table rows Unit and Mapping);
+* a fresh block is taken from one global free pool only when the sequence's last
+  block is full ("How it works -- The mechanics"; lesson: "allocate a new block
+  only when decode fills the last one"), so the waste is at most one partly
+  filled block per sequence;
+* a finished sequence frees its blocks and they go back to the pool;
+* sequences that share content point their tables at the same physical blocks,
+  with a reference count, and a block is copied only when a sequence writes
+  into it while it is shared (ops page, How it works and At a glance).
+
+Readings where the pages are silent (fixed only so that two implementations
+can be compared exactly; any order is correct by the pages):
+
+* the free pool is a LIFO stack; it starts holding ``free_order`` with
+  ``free_order[0]`` on top (default ``0, 1, 2, ...``);
+* a freed sequence pushes its blocks in logical order, so its last block ends on
+  top and is the next one handed out; shared blocks are only decremented;
+* sequence ids count up from 0 and are never reused;
+* ``reserve`` is all-or-nothing: if the pool cannot cover every block it needs
+  (copy included) it changes nothing and reports exhaustion;
+* ``cow(seq, i)`` gives the sequence a private copy of logical block i when the
+  block is shared, and does nothing otherwise;
+* a slot id is ``physical_block * block_size + offset``.
+"""
+
+from __future__ import annotations
+
+
+class PoolExhausted(Exception):
+    """The free pool cannot cover the request (the pages' trigger for preemption)."""
+
+
+class BlockPoolModel:
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        if num_blocks <= 0 or block_size <= 0:
+            raise ValueError("num_blocks and block_size must be positive")
+        self.num_blocks = int(num_blocks)
+        self.block_size = int(block_size)
+        order = list(range(num_blocks)) if free_order is None else [int(x) for x in free_order]
+        if sorted(order) != list(range(num_blocks)):
+            raise ValueError("free_order must be a permutation of the block ids")
+        # The stack's top is the end of the list.
+        self.free = list(reversed(order))
+        self.refcount = [0] * self.num_blocks
+        self.seqs = {}  # id -> {"blocks": [phys ids], "len": tokens}
+        self.next_id = 0
+
+    # -- sequences -----------------------------------------------------------
+    def new_seq(self) -> int:
+        sid = self.next_id
+        self.next_id += 1
+        self.seqs[sid] = {"blocks": [], "len": 0}
+        return sid
+
+    def fork(self, parent: int) -> int:
+        """A new sequence that shares every block of ``parent`` (refcount + 1 each)."""
+        src = self.seqs[parent]
+        sid = self.new_seq()
+        self.seqs[sid]["blocks"] = list(src["blocks"])
+        self.seqs[sid]["len"] = src["len"]
+        for b in src["blocks"]:
+            self.refcount[b] += 1
+        return sid
+
+    def _pop(self) -> int:
+        b = self.free.pop()
+        self.refcount[b] = 1
+        return b
+
+    def reserve(self, sid: int, n_tokens: int):
+        """Make room for ``n_tokens`` more tokens; return (slots, cow_pairs)."""
+        seq = self.seqs[sid]
+        bs = self.block_size
+        length = seq["len"]
+        # Count what the request needs before touching anything.
+        need = 0
+        pos = length
+        for _ in range(n_tokens):
+            if pos % bs == 0:
+                need += 1
+            pos += 1
+        cow_needed = (n_tokens > 0 and length % bs != 0
+                      and self.refcount[seq["blocks"][length // bs]] > 1)
+        if cow_needed:
+            need += 1
+        if need > len(self.free):
+            raise PoolExhausted(f"need {need} blocks, {len(self.free)} free")
+
+        slots, pairs = [], []
+        for _ in range(n_tokens):
+            pos = seq["len"]
+            if pos % bs == 0:
+                # The last block is full (or there is none): take a fresh one.
+                seq["blocks"].append(self._pop())
+            else:
+                cur = seq["blocks"][pos // bs]
+                if self.refcount[cur] > 1:
+                    # Writing into a shared block: copy it first.
+                    fresh = self._pop()
+                    self.refcount[cur] -= 1
+                    seq["blocks"][pos // bs] = fresh
+                    pairs.append((cur, fresh))
+            slots.append(seq["blocks"][pos // bs] * bs + pos % bs)
+            seq["len"] = pos + 1
+        return slots, pairs
+
+    def cow(self, sid: int, logical_block: int):
+        """Give ``sid`` a private copy of one shared block; return the pair or None."""
+        seq = self.seqs[sid]
+        cur = seq["blocks"][logical_block]
+        if self.refcount[cur] <= 1:
+            return None
+        if not self.free:
+            raise PoolExhausted("no free block for the copy")
+        fresh = self._pop()
+        self.refcount[cur] -= 1
+        seq["blocks"][logical_block] = fresh
+        return (cur, fresh)
+
+    def free_seq(self, sid: int) -> None:
+        seq = self.seqs.pop(sid)
+        for b in seq["blocks"]:
+            self.refcount[b] -= 1
+            if self.refcount[b] == 0:
+                self.free.append(b)
+
+    # -- views ---------------------------------------------------------------
+    def table(self, sid: int):
+        return list(self.seqs[sid]["blocks"])
+
+    def length(self, sid: int) -> int:
+        return self.seqs[sid]["len"]
+
+    def free_list(self):
+        """Free ids from the top of the stack down (next to be handed out first)."""
+        return list(reversed(self.free))
+
+    def stats(self) -> dict:
+        bs = self.block_size
+        live = set()
+        for seq in self.seqs.values():
+            for t in range(seq["len"]):
+                live.add((seq["blocks"][t // bs], t % bs))
+        allocated = self.num_blocks - len(self.free)
+        return {
+            "free_blocks": len(self.free),
+            "allocated_slots": allocated * bs,
+            "live_slots": len(live),
+            "live_tokens": sum(s["len"] for s in self.seqs.values()),
+            "shared_blocks": sum(1 for r in self.refcount if r > 1),
+            "num_seqs": len(self.seqs),
+        }
+
+
+def contiguous_reservation_waste(lengths, reserve_tokens: int) -> dict:
+    """The slab scheme the pages compare against: every request reserves
+    ``reserve_tokens`` contiguous slots up front ("PagedAttention" ops page,
+    Concept -- What it is; KV-cache lesson, problem statement)."""
+    reserved = reserve_tokens * len(lengths)
+    live = sum(min(int(x), reserve_tokens) for x in lengths)
+    return {"reserved_slots": reserved, "live_slots": live, "wasted_slots": reserved - live}
