@@ -1,0 +1,521 @@
+"""Benchmark of the paged decode step on B200: append + copy-on-write + decode.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch: the new token of every
+sequence is appended through its slot (plus the block copies when the workload
+shares blocks), then every sequence's query attends over its context through the
+block table.  Inputs are resident in HBM before the timed region; the step is
+replayed from two CUDA graphs (append+copy, decode) with CUDA events between them
+on the launching stream.  The KV read per step (554 MB at the default workload)
+is 4x the 126 MB L2, so L2 is not flushed between steps.
+
+Multi-GPU (torchrun): each rank runs its own seeded batch (weak scaling, no
+collective on the data path); times are the max over ranks.
+
+``--impl reference`` times the CPU oracle on the host cores instead (bounded
+samples of the same workload); under torchrun only rank 0 runs it.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV GB/s (% of B200 HBM peak); seq-decode-steps/sec"
+FALLBACK_HBM_GBS = 6650.0
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+# ---------------------------------------------------------------- accounting
+
+def decode_bytes(lens, wl) -> int:
+    """Algorithmic bytes of one decode: K and V of every live token once, q, out,
+    the block-table entries read and the lengths."""
+    es = 2
+    kv = int(np.sum(lens, dtype=np.int64)) * wl.num_kv_heads * wl.head_dim * es * 2
+    qo = 2 * wl.num_seqs * wl.num_heads * wl.head_dim * es
+    table = int(np.sum((np.asarray(lens, dtype=np.int64) + wl.block_size - 1) // wl.block_size)) * 4
+    return kv + qo + table + 4 * wl.num_seqs
+
+
+def append_bytes(n_tokens, wl) -> int:
+    row = wl.num_kv_heads * wl.head_dim * 2
+    return n_tokens * (2 * row * 2 + 8)        # read key+value, write them, read the slot
+
+
+def copy_bytes(n_pairs, wl) -> int:
+    block = wl.num_kv_heads * wl.block_size * wl.head_dim * 2
+    return n_pairs * (2 * 2 * block + 8)       # K and V: read + write, read the pair
+
+
+# --------------------------------------------------------------- multi-rank
+
+def max_over_ranks(values, world, device=None):
+    """Max of each value over all ranks (device times: the slowest rank decides)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_gbs(bytes_per_rank_step, world, ms_per_step) -> float:
+    """Aggregate throughput: every rank processes its own batch in the same step time."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
+# ------------------------------------------------------------------ workload
+
+def build_step(wl, pkv):
+    """Host bookkeeping for one decode step with the library's block manager.
+
+    Returns (pairs, slots, tables, lens, key, value): the copy pairs, the slots
+    of the appended tokens, the block tables and lengths the decode reads, and
+    the keys/values appended."""
+    bs = wl.block_size
+    pool = pkv.Pool(wl.num_blocks, bs, wl.free_order)
+    pairs, slots = [], []
+    if wl.prefix_len:
+        s0 = pool.new_seq()
+        pool.reserve(s0, wl.prefix_len)
+        seqs = [s0] + [pool.fork(s0) for _ in range(wl.num_seqs - 1)]
+        last_prefix_block = (wl.prefix_len + bs - 1) // bs - 1
+        for s in seqs:
+            p = pool.cow(s, last_prefix_block)
+            if p:
+                pairs.append(p)
+        for b, s in enumerate(seqs):
+            sl, cp = pool.reserve(s, int(wl.suffix_lens[b]) + 1)
+            pairs.extend(cp)
+            slots.extend(int(x) for x in sl)
+    else:
+        seqs = []
+        for b in range(wl.num_seqs):
+            s = pool.new_seq()
+            pool.reserve(s, int(wl.context_lens[b]) - 1)
+            seqs.append(s)
+        for s in seqs:
+            sl, cp = pool.reserve(s, 1)
+            pairs.extend(cp)
+            slots.extend(int(x) for x in sl)
+    mb = max(len(pool.table(s)) for s in seqs)
+    tables, lens = pool.block_tables(seqs, mb, pad=-1)
+    pool.close()
+    return (np.array(pairs, dtype=np.int32).reshape(-1, 2), np.array(slots, dtype=np.int64),
+            tables, lens, wl.new_key, wl.new_value)
+
+
+# ------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    def __init__(self, period_ms=20):
+        self.period_ms = period_ms
+        self.rows = []
+        self.proc = None
+        self.marks = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                 f"-lms={self.period_ms}"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def mark(self, name):
+        self.marks.append((name, time.time()))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        inside = [r for t, r in self.rows if t0 <= t <= t1]
+        window = "timed region"
+        if len(inside) < 3:
+            inside = [r for t, r in self.rows]
+            window = "whole run (timed region shorter than the sampling period)"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in inside if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in inside if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i in range(4)
+                          if len(r) > 5 + i and r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(inside), "window": window}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_record():
+    """DRAM bytes per decode launch from the committed ncu summary
+    profiles/decode_traffic.txt, if it was taken on the current decode source
+    (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "decode_traffic.txt")
+    try:
+        rec = {}
+        for line in open(path):
+            if ":" in line and not line.startswith("#"):
+                key, val = line.split(":", 1)
+                rec[key.strip()] = val.strip()
+    except OSError:
+        return None
+    src = open(os.path.join(ROOT, "paged_kv_cache_360_b200", "csrc", "pkv_decode.cu"), "rb").read()
+    if rec.get("source_sha256") != hashlib.sha256(src).hexdigest():
+        return None
+    return {"bytes_per_launch": int(rec["bytes_per_launch"])}
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import paged_kv_cache_360_b200 as pkv
+    from paged_kv_cache_360_b200.workloads import make_workload
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = make_workload(args.config, seed=args.seed, rank=rank)
+    pairs, slots, tables, lens, new_key, new_value = build_step(wl, pkv)
+
+    k = wl.k_cache.to(dev)
+    v = wl.v_cache.to(dev)
+    q = wl.q.to(dev)
+    d_key, d_value = new_key.to(dev), new_value.to(dev)
+    d_slots = torch.from_numpy(slots).to(dev)
+    d_pairs = torch.from_numpy(pairs).to(dev)
+    d_tables = torch.from_numpy(tables).to(dev)
+    d_lens = torch.from_numpy(lens).to(dev)
+    out = torch.empty_like(q)
+    B, H = wl.num_seqs, wl.num_heads
+    P = wl.partition_size or pkv.paged_attention_partition_size(k, B, H, tables.shape[1])
+    ws_bytes = pkv.paged_attention_workspace_bytes(k, B, H, tables.shape[1], P)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step_write():
+        if len(pairs):
+            pkv.copy_blocks(k, v, d_pairs, err_flag=err)
+        pkv.paged_kv_append(k, v, d_key, d_value, d_slots, err_flag=err)
+
+    def step_decode():
+        pkv.paged_attention_decode(out, q, k, v, d_tables, d_lens, wl.scale, partition_size=P,
+                                   workspace=ws, err_flag=err)
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        n0 = pkv.launch_count()
+        step_write()
+        step_decode()
+        launches_per_step = pkv.launch_count() - n0
+    torch.cuda.synchronize()
+    g_write, g_decode = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_write, stream=stream):
+        step_write()
+    with torch.cuda.graph(g_decode, stream=stream):
+        step_decode()
+    torch.cuda.synchronize()
+
+    step_bytes_decode = decode_bytes(lens, wl)
+    step_bytes = step_bytes_decode + append_bytes(len(slots), wl) + copy_bytes(len(pairs), wl)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    sampler = ClockSampler()
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            g_write.replay()
+            g_decode.replay()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            g_write.replay()
+            evs[i][1].record(stream)
+            g_decode.replay()
+            evs[i][2].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    step_ms = sum(e[0].elapsed_time(e[2]) for e in evs)
+    decode_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+
+    # end to end through the public API: pinned host inputs -> device -> kernels -> host
+    h = {name: t.pin_memory() for name, t in (("q", wl.q), ("key", new_key), ("value", new_value),
+                                               ("slots", torch.from_numpy(slots)),
+                                               ("tables", torch.from_numpy(tables)),
+                                               ("lens", torch.from_numpy(lens)))}
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dst = {"q": q, "key": d_key, "value": d_value, "slots": d_slots, "tables": d_tables, "lens": d_lens}
+    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    d2h = h_out.numel() * h_out.element_size()
+    e2e_steps = max(3, min(args.steps, 200))
+    e2e_ms = 0.0
+    barrier()
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup + e2e_steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for name, t in h.items():
+                dst[name].copy_(t, non_blocking=True)
+            step_write()
+            step_decode()
+            h_out.copy_(out, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            if i >= args.warmup:
+                e2e_ms += e0.elapsed_time(e1)
+    barrier()
+    if rank == 0:
+        sampler.stop()
+    torch.cuda.synchronize()
+    err_val = int(err.item())
+
+    step_ms, decode_ms, e2e_ms = max_over_ranks([step_ms, decode_ms, e2e_ms], world, dev)
+    if rank != 0:
+        return None
+
+    peak, peak_kind = measured_peak()
+    ms_per_step = step_ms / args.steps
+    value = whole_job_gbs(step_bytes, world, ms_per_step)
+    decode_avg_ms = decode_ms / args.steps
+    achieved = step_bytes_decode / (decode_avg_ms * 1e-3) / 1e9
+    traffic = traffic_record()
+    e2e_per_step = e2e_ms / e2e_steps
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "num_seqs_per_gpu": B, "global_num_seqs": B * world,
+                   "num_heads": H, "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+                   "block_size": wl.block_size, "num_blocks": wl.num_blocks,
+                   "mean_context_len": float(np.mean(lens)), "max_context_len": int(np.max(lens)),
+                   "partition_size": int(P), "copy_pairs": int(len(pairs)),
+                   "appended_tokens": int(len(slots)), "seed": args.seed,
+                   "parallelism": f"dp{world} (independent batches per GPU)",
+                   "l2": "not flushed: the step reads %.0f MB of K/V, %.1fx the 126 MB L2"
+                         % (step_bytes_decode / 1e6, step_bytes_decode / 126e6),
+                   "timing": "CUDA events around CUDA-graph replays of the step on its stream"},
+        "seq_decode_steps_per_s": round(world * B / (ms_per_step * 1e-3), 1),
+        "hbm_frac": round(value / world / peak, 4),
+        "algorithmic_bytes_per_step": step_bytes,
+        "roofline": {"bound": "hbm", "kernel": "paged_attention_decode (partition + reduce kernels)",
+                     "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": None if traffic is None else traffic["bytes_per_launch"],
+                     "algorithmic_bytes_per_launch": step_bytes_decode,
+                     "avg_launch_ms": round(decode_avg_ms, 5)},
+        "e2e": {"value": round(whole_job_gbs(step_bytes, world, e2e_per_step), 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_per_step, 5), "steps": e2e_steps,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "path": "pinned host -> device copies, paged_kv_append, paged_attention_decode, "
+                        "device -> pinned host, all on one stream, eager"},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "launches_per_step": int(launches_per_step),
+        "device_err_flag": err_val,
+        "clocks": sampler.summary(t_wall0, t_wall1),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, lens, tables, slots, new_key, new_value,
+                                            budget_s=args.cpu_budget)
+    return line
+
+
+# ------------------------------------------------------ CPU oracle (baseline)
+
+def sample_bytes(wl, sub_lens, n) -> int:
+    """Algorithmic bytes of an oracle sample: n whole sequences decoded (plus
+    their appended tokens when the workload appends one per sequence)."""
+    es = 2
+    sub = np.asarray(sub_lens, dtype=np.int64)
+    return int(sub.sum()) * wl.num_kv_heads * wl.head_dim * es * 2 + \
+        2 * n * wl.num_heads * wl.head_dim * es + \
+        int(np.sum((sub + wl.block_size - 1) // wl.block_size)) * 4 + 4 * n + \
+        (0 if wl.prefix_len else append_bytes(n, wl))
+
+
+def _oracle_sample(wl, tables, lens, slots, key, value, seqs):
+    """Oracle append of the sample's new tokens, then oracle decode of the sample."""
+    import oracle
+    kw, vw = oracle.words(wl.k_cache), oracle.words(wl.v_cache)
+    if not wl.prefix_len:
+        idx = np.asarray(seqs)
+        oracle.append(kw, vw, key[idx], value[idx], slots[idx])
+    t = np.ascontiguousarray(tables[seqs])
+    l = np.ascontiguousarray(lens[seqs])
+    return oracle.paged_decode(wl.q[seqs], kw, vw, t, l, wl.scale)
+
+
+def cpu_baseline(wl, lens, tables, slots, key, value, budget_s=12.0):
+    """Time the oracle (single-threaded C, float64) on a bounded sample: whole
+    sequences of the same batch, in order, until about `budget_s` of CPU time."""
+    import oracle
+    oracle.build()
+    # calibrate on the first sequence
+    t0 = time.perf_counter()
+    _oracle_sample(wl, tables, lens, slots, key, value, [0])
+    per_token = (time.perf_counter() - t0) / max(1, int(lens[0]))
+    n, tokens = 0, 0
+    while n < wl.num_seqs and (tokens + int(lens[n])) * per_token < budget_s:
+        tokens += int(lens[n])
+        n += 1
+    n = max(n, 1)
+    seqs = list(range(n))
+    t0 = time.perf_counter()
+    _oracle_sample(wl, tables, lens, slots, key, value, seqs)
+    dt = time.perf_counter() - t0
+    sub_lens = lens[:n]
+    nbytes = sample_bytes(wl, sub_lens, n)
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle", "seconds": round(dt, 3),
+            "seq_decode_steps_per_s": round(n / dt, 3),
+            "sample": f"first {n} of {wl.num_seqs} sequences of the {wl.name} batch "
+                      f"({int(np.sum(sub_lens))} context tokens): oracle append + decode, 1 pass, "
+                      f"single-threaded C float64 on {os.cpu_count()} host cores available"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    from paged_kv_cache_360_b200.workloads import make_workload
+    import oracle
+    import paged_kv_cache_360_b200 as pkv
+    oracle.build()
+    wl = make_workload(args.config, seed=args.seed, rank=0)
+    pairs, slots, tables, lens, key, value = build_step(wl, pkv)
+    budget = args.ref_step_budget
+    t0 = time.perf_counter()
+    _oracle_sample(wl, tables, lens, slots, key, value, [0])
+    per_token = (time.perf_counter() - t0) / max(1, int(lens[0]))
+    n, tokens = 0, 0
+    while n < wl.num_seqs and (tokens + int(lens[n])) * per_token < budget:
+        tokens += int(lens[n])
+        n += 1
+    n = max(n, 1)
+    seqs = list(range(n))
+    for _ in range(args.warmup):
+        _oracle_sample(wl, tables, lens, slots, key, value, seqs)
+    total = 0.0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        _oracle_sample(wl, tables, lens, slots, key, value, seqs)
+        total += time.perf_counter() - t0
+    sub_lens = lens[:n]
+    nbytes = sample_bytes(wl, sub_lens, n)
+    ms = total / args.steps * 1e3
+    value_gbs = nbytes / (ms * 1e-3) / 1e9
+    sample = (f"each step: first {n} of {wl.num_seqs} sequences of the {wl.name} batch "
+              f"({int(np.sum(sub_lens))} context tokens), oracle append + decode, single-threaded C float64")
+    return {"impl": "reference", "metric": METRIC, "value": round(value_gbs, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "num_seqs_sampled": n, "num_heads": wl.num_heads,
+                       "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+                       "block_size": wl.block_size, "seed": args.seed},
+            "seq_decode_steps_per_s": round(n / (ms * 1e-3), 3),
+            "cpu_baseline": {"value": round(value_gbs, 4), "unit": "GB/s", "cores": 1,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value_gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU time")
+    ap.add_argument("--ref-step-budget", type=float, default=3.0,
+                    help="seconds of oracle CPU time per reference step")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            ap.error("--gpus N > 1 must be launched with torchrun (one process per GPU)")
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,261 @@
+/*
+ * pkv.h -- C ABI of libpkv, paged KV-cache decode attention for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow three web pages on PagedAttention:
+ *   [ops page]  "PagedAttention" operations page (foundry.adhana.ai), sections
+ *               "Concept -- What it is" and "How it works -- The mechanics";
+ *   [lesson]    "Paged Attention", lesson 3 of "The KV Cache" (aiacademy.guru),
+ *               the method paragraph and the virtual-memory analogy table;
+ *   [glossary]  "PagedAttention" glossary entry (aimodelwiki.com).
+ * The pages fix the data structures (fixed-size KV blocks in one pool, a block
+ * table per sequence, a free pool, reference-counted sharing with copy on write)
+ * and the fact that the attention kernel gathers K/V through the block table.
+ * They fix no API, layout or precision; those choices are stated here.
+ *
+ * Conventions for every call below
+ * --------------------------------
+ * - Layout.  A cache pool is [num_blocks][num_kv_heads][block_size][head_dim]
+ *   elements of `dtype`, row-major; K and V are two pools of the same shape.  A
+ *   slot id is `block * block_size + offset`.  q and out are [num_seqs][num_heads]
+ *   [head_dim]; query head h reads kv head h / (num_heads / num_kv_heads).
+ * - Ownership.  Every device buffer (pools, q, out, tables, lengths, slot and
+ *   copy lists, workspace, err_flag) belongs to the caller.  The device calls
+ *   allocate no device memory and keep no state between calls.
+ * - Pointers.  "device" pointers must be device-accessible CUDA allocations on
+ *   the current device; "host" pointers are ordinary host memory.
+ * - Streams.  `stream` is a cudaStream_t (passed as void*; NULL = legacy default
+ *   stream).  Device calls are asynchronous and stream-ordered: they validate
+ *   their host-side arguments, enqueue kernels and return.
+ * - Errors.  Host-side validation fails before anything is enqueued and returns
+ *   PKV_ERR_INVALID_ARG / PKV_ERR_UNSUPPORTED / PKV_ERR_WORKSPACE_TOO_SMALL.  A
+ *   failed launch returns PKV_ERR_CUDA.  Device-side checks (a block id outside
+ *   the pool, a context length beyond the table, a slot past the pool) never
+ *   trap: the kernel ORs a PKV_DEVERR_* bit into `*err_flag` (device int32,
+ *   optional, the caller clears it) and skips or clamps the offending access.
+ *   pkv_last_error() gives a message for the last failing call of this thread.
+ * - Supported shapes.  head_dim in {64, 128}; block_size in {16, 32}; dtype
+ *   fp16 or bf16; 1 <= num_heads / num_kv_heads <= 16; num_blocks * num_kv_heads
+ *   * block_size < 2^31.  Others return PKV_ERR_UNSUPPORTED.
+ */
+#ifndef PKV_H_
+#define PKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pkv_status {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = 1,         /* null / misaligned pointer, bad count or id     */
+    PKV_ERR_UNSUPPORTED = 2,         /* shape or dtype outside the supported set       */
+    PKV_ERR_NO_FREE_BLOCK = 3,       /* the free pool cannot cover the request         */
+    PKV_ERR_CUDA = 4,                /* a CUDA call or kernel launch failed            */
+    PKV_ERR_WORKSPACE_TOO_SMALL = 5  /* decode workspace smaller than required         */
+} pkv_status;
+
+typedef enum pkv_dtype { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
+
+/* Bits a kernel ORs into *err_flag. */
+#define PKV_DEVERR_BAD_BLOCK_ID 1    /* table entry outside [0, num_blocks): block 0 read instead */
+#define PKV_DEVERR_BAD_CONTEXT_LEN 2 /* context length < 0 or > max_blocks_per_seq*block_size: clamped */
+#define PKV_DEVERR_BAD_SLOT 4        /* slot >= num_blocks*block_size: token skipped */
+#define PKV_DEVERR_WAIT_TIMEOUT 8    /* a pipeline wait ran past its iteration limit: work skipped */
+#define PKV_DEVERR_BAD_PAIR 16       /* copy pair id outside the pool: pair skipped */
+
+/* Shape of one KV pool (shared by the K and V pools). */
+typedef struct pkv_cache_desc {
+    int32_t num_blocks;   /* physical blocks in the pool                    */
+    int32_t block_size;   /* tokens per block (16 or 32)                    */
+    int32_t num_kv_heads; /* key/value heads                                */
+    int32_t head_dim;     /* elements per head (64 or 128)                  */
+    pkv_dtype dtype;      /* element type of q, out, pools, key, value      */
+} pkv_cache_desc;
+
+/* ------------------------------------------------------------- device calls */
+
+/*
+ * Append: write the keys and values of num_tokens new tokens into the pools
+ * through a slot mapping ([ops page] How it works: each decode step writes the
+ * new token's key and value into the sequence's current block; [lesson]
+ * analogy table, Allocation row).
+ *   k_cache, v_cache  device, pools as above, written in place.
+ *   key, value        device, [num_tokens][num_kv_heads][head_dim], 16-byte aligned.
+ *   slot_mapping      device int64 [num_tokens]; token i goes to slot
+ *                     slot_mapping[i]; a negative slot skips the token (padding).
+ *                     Slots must be distinct (duplicates: unspecified winner).
+ *   err_flag          device int32 or NULL; PKV_DEVERR_BAD_SLOT for a slot past the pool.
+ * num_tokens == 0 enqueues nothing.  Bit-exact copy of the input rows.
+ */
+pkv_status paged_kv_append(const pkv_cache_desc* desc, void* k_cache, void* v_cache,
+                           const void* key, const void* value, const int64_t* slot_mapping,
+                           int32_t num_tokens, int32_t* err_flag, void* stream);
+
+/*
+ * Copy-on-write block copy: for each pair (src, dst) copy block src over block
+ * dst -- every kv head and offset -- in both pools ([ops page] How it works:
+ * sequences that share blocks "only copy-on-write when they diverge"; At a
+ * glance: a block is copied only when a sequence writes to it).
+ *   block_mapping  device int32 [num_pairs][2] = (src, dst).  Destinations must
+ *                  be distinct and no destination may be a source (pairs run
+ *                  concurrently); the host block manager's pairs always are.
+ *   err_flag       device int32 or NULL; PKV_DEVERR_BAD_PAIR for an id outside the pool.
+ * num_pairs == 0 enqueues nothing.  Bit-exact.
+ */
+pkv_status copy_blocks(const pkv_cache_desc* desc, void* k_cache, void* v_cache,
+                       const int32_t* block_mapping, int32_t num_pairs, int32_t* err_flag,
+                       void* stream);
+
+/*
+ * Partition size (tokens) the decode uses when called with partition_size 0:
+ * 0 means "one pass per (sequence, kv head), no split"; otherwise a multiple of
+ * block_size.  Depends only on the arguments and the current device's SM count.
+ */
+int32_t paged_attention_partition_size(const pkv_cache_desc* desc, int32_t num_seqs,
+                                       int32_t num_heads, int32_t max_blocks_per_seq);
+
+/*
+ * Workspace bytes paged_attention_decode needs for these shapes and
+ * partition_size (0 = the library's choice above).  0 when no split is used.
+ * Layout (float32): partial outputs [num_seqs][num_heads][P_max][head_dim], then
+ * maxima and sums [num_seqs][num_heads][P_max] each, with
+ * P_max = ceil(max_blocks_per_seq * block_size / partition_size).
+ */
+size_t paged_attention_workspace_bytes(const pkv_cache_desc* desc, int32_t num_seqs,
+                                       int32_t num_heads, int32_t max_blocks_per_seq,
+                                       int32_t partition_size);
+
+/*
+ * Paged decode attention: one query token per sequence attends over its
+ * context, reading keys and values through the block table ([ops page] How it
+ * works: the kernel "reads KV through the block table, gathering scattered
+ * physical blocks"; Concept: the block table maps logical positions to
+ * physical blocks; [glossary]).
+ *   out[b][h][:] = sum_t softmax_t(scale * q[b][h] . K[b][t]) V[b][t],
+ *   t < context_lens[b], K/V of logical token t read from physical block
+ *   block_tables[b][t / block_size] at offset t % block_size, kv head
+ *   h / (num_heads / num_kv_heads).
+ * Arithmetic: fp16/bf16 inputs, fp32 scores, softmax and accumulation, the
+ * probabilities rounded to `dtype` for the probability-value product, output
+ * rounded to `dtype`.  The reduction order depends only on logical token order,
+ * so the result is bit-identical under any permutation of physical blocks.
+ *   out, q          device [num_seqs][num_heads][head_dim], 16-byte aligned.
+ *   k_cache, v_cache device pools, 16-byte aligned (read only).
+ *   block_tables    device int32 [num_seqs][max_blocks_per_seq]; entries at or
+ *                   past ceil(context_len / block_size) are not read.
+ *   context_lens    device int32 [num_seqs]; 0 gives an output of zeros.
+ *   partition_size  0 = library's choice; otherwise a multiple of block_size;
+ *                   sequences longer than it are split into partitions whose
+ *                   partial results a second kernel merges by log-sum-exp.
+ *   workspace       device, >= paged_attention_workspace_bytes(...), 16-byte
+ *                   aligned; may be NULL when that size is 0.
+ *   err_flag        device int32 or NULL (PKV_DEVERR_BAD_BLOCK_ID,
+ *                   PKV_DEVERR_BAD_CONTEXT_LEN, PKV_DEVERR_WAIT_TIMEOUT).
+ */
+pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* out, const void* q,
+                                  const void* k_cache, const void* v_cache,
+                                  const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t* context_lens, int32_t num_seqs,
+                                  int32_t num_heads, float scale, int32_t partition_size,
+                                  void* workspace, size_t workspace_bytes, int32_t* err_flag,
+                                  void* stream);
+
+/* -------------------------------------------------- host block bookkeeping */
+/*
+ * The block manager of [ops page] Concept and How it works and the [lesson]
+ * analogy table: a pool of num_blocks fixed-size blocks, one free pool, a block
+ * table per sequence, blocks handed out one at a time when the last one fills,
+ * freed blocks returned to the pool, sharing by reference count (fork) and copy
+ * on write.  Host memory only; not thread-safe (one pool per thread, or lock).
+ * Tie-breaks the pages leave open, fixed so results are reproducible:
+ *   - the free pool is a LIFO stack that starts with free_order[0] on top
+ *     (free_order NULL = 0, 1, 2, ...);
+ *   - pkv_seq_free pushes a sequence's blocks in logical order (its last block
+ *     ends on top); shared blocks are only decremented;
+ *   - sequence ids count up from 0 and are never reused;
+ *   - a request that the free pool cannot cover fails with
+ *     PKV_ERR_NO_FREE_BLOCK and changes nothing.
+ */
+typedef struct pkv_pool pkv_pool;
+
+typedef struct pkv_stats {
+    int64_t free_blocks;     /* blocks in the free pool                              */
+    int64_t allocated_slots; /* (num_blocks - free_blocks) * block_size              */
+    int64_t live_slots;      /* distinct slots holding a token of a live sequence    */
+    int64_t live_tokens;     /* sum of live sequence lengths (shared tokens counted per sequence) */
+    int64_t shared_blocks;   /* blocks with reference count > 1                      */
+    int64_t num_seqs;        /* live sequences                                       */
+} pkv_stats;
+
+/* free_order: host int32 [num_blocks], a permutation of 0..num_blocks-1, or NULL. */
+pkv_status pkv_pool_create(int32_t num_blocks, int32_t block_size, const int32_t* free_order,
+                           pkv_pool** out);
+void pkv_pool_destroy(pkv_pool* pool);
+
+/* A new, empty sequence. */
+pkv_status pkv_seq_new(pkv_pool* pool, int32_t* seq_id);
+
+/* A new sequence sharing every block of `parent` (each block's refcount + 1). */
+pkv_status pkv_seq_fork(pkv_pool* pool, int32_t parent, int32_t* child);
+
+/*
+ * Make room for n_tokens more tokens of `seq`: slots_out (host int64
+ * [n_tokens]) receives their slot ids in order.  A fresh block is taken only
+ * when the last block is full.  If the first token lands in a partly filled
+ * block that other sequences share, that block is first copied: the pair
+ * (src, dst) goes to cow_pair_out (host int32 [2]) and *n_cow_out is 1, else 0.
+ * The caller must run copy_blocks on the pair before appending.
+ */
+pkv_status pkv_seq_reserve(pkv_pool* pool, int32_t seq, int32_t n_tokens, int64_t* slots_out,
+                           int32_t* cow_pair_out, int32_t* n_cow_out);
+
+/*
+ * Give `seq` a private copy of its logical block `logical_block` if that block
+ * is shared: the pair goes to pair_out (host int32 [2]), *n_out = 1; a block
+ * already private gives *n_out = 0.
+ */
+pkv_status pkv_seq_cow(pkv_pool* pool, int32_t seq, int32_t logical_block, int32_t* pair_out,
+                       int32_t* n_out);
+
+/* Release the sequence: every block's refcount - 1; blocks reaching 0 return to the pool. */
+pkv_status pkv_seq_free(pkv_pool* pool, int32_t seq);
+
+pkv_status pkv_seq_len(const pkv_pool* pool, int32_t seq, int64_t* len);
+
+/* The sequence's block table: *n entries, at most cap of them written to row. */
+pkv_status pkv_seq_block_table(const pkv_pool* pool, int32_t seq, int32_t* row, int32_t cap,
+                               int32_t* n);
+
+/*
+ * Decode-step export: for the n_seqs sequences listed in seqs, write their
+ * block tables into tables (host int32 [n_seqs][max_blocks_per_seq], unused
+ * entries set to pad) and their lengths into context_lens (host int32 [n_seqs]).
+ */
+pkv_status pkv_pool_block_tables(const pkv_pool* pool, const int32_t* seqs, int32_t n_seqs,
+                                 int32_t* tables, int32_t max_blocks_per_seq,
+                                 int32_t* context_lens, int32_t pad);
+
+pkv_status pkv_pool_refcount(const pkv_pool* pool, int32_t block, int32_t* refcount);
+
+/* Free ids from the top of the stack down: *n entries, at most cap written. */
+pkv_status pkv_pool_free_list(const pkv_pool* pool, int32_t* out, int32_t cap, int32_t* n);
+
+pkv_status pkv_pool_stats(const pkv_pool* pool, pkv_stats* stats);
+
+/* --------------------------------------------------------------- diagnostics */
+
+/* Kernels this library has launched in this process (all devices, all threads). */
+uint64_t pkv_launch_count(void);
+
+/* Message for the last non-OK status returned to this thread ("" if none). */
+const char* pkv_last_error(void);
+
+const char* pkv_status_string(pkv_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H_ */

@@ -1,0 +1,232 @@
+"""Paged KV-cache decode attention for NVIDIA B200 (sm_100a).
+
+A thin Python binding over libpkv.so (include/pkv.h): the functions below have
+the C ABI's names and only marshal arguments -- tensor pointers, shapes and the
+current CUDA stream.  Every step runs in the library's CUDA kernels or its C++
+block manager; there is no CPU fallback.  Device calls require CUDA tensors and
+raise if the library is not built.
+
+PyTorch provides device memory and streams only.
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import _lib
+from ._lib import PkvError, PoolExhausted  # noqa: F401
+
+__all__ = [
+    "paged_kv_append", "copy_blocks", "paged_attention_decode", "paged_attention_workspace_bytes",
+    "paged_attention_partition_size", "Pool", "PkvError", "PoolExhausted", "launch_count",
+    "cache_desc",
+]
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return _lib.PKV_BF16
+    if t.dtype == torch.float16:
+        return _lib.PKV_F16
+    raise PkvError(2, f"unsupported dtype {t.dtype}: fp16 or bf16 only")
+
+
+def cache_desc(k_cache) -> _lib.CacheDesc:
+    """Descriptor of a pool tensor [num_blocks, num_kv_heads, block_size, head_dim]."""
+    if k_cache.dim() != 4:
+        raise PkvError(1, "cache must be [num_blocks, num_kv_heads, block_size, head_dim]")
+    nb, hkv, bs, d = k_cache.shape
+    return _lib.CacheDesc(nb, bs, hkv, d, _dtype_code(k_cache))
+
+
+def _dev(t, name: str, dtype=None):
+    """Device pointer of a contiguous CUDA tensor (raises otherwise)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise PkvError(1, f"{name} must be a CUDA tensor (this library has no CPU path)")
+    if not t.is_contiguous():
+        raise PkvError(1, f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise PkvError(1, f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = _torch().cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def paged_kv_append(k_cache, v_cache, key, value, slot_mapping, err_flag=None, stream=None):
+    """Write key/value [N, Hkv, D] into the pools at slot_mapping (int64 [N]; < 0 skips)."""
+    torch = _torch()
+    desc = cache_desc(k_cache)
+    if tuple(key.shape) != (slot_mapping.shape[0], k_cache.shape[1], k_cache.shape[3]) or \
+            key.shape != value.shape or key.dtype != k_cache.dtype or value.dtype != k_cache.dtype:
+        raise PkvError(1, "key/value must be [N, num_kv_heads, head_dim] of the cache dtype")
+    _lib.check(_lib.load().paged_kv_append(
+        ctypes.byref(desc), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), _dev(key, "key"),
+        _dev(value, "value"), _dev(slot_mapping, "slot_mapping", torch.int64),
+        int(slot_mapping.shape[0]), _dev(err_flag, "err_flag", torch.int32), _stream(stream)))
+
+
+def copy_blocks(k_cache, v_cache, block_mapping, err_flag=None, stream=None):
+    """Copy whole blocks src -> dst for each row (src, dst) of block_mapping (int32 [M, 2])."""
+    torch = _torch()
+    desc = cache_desc(k_cache)
+    if block_mapping.dim() != 2 or block_mapping.shape[1] != 2:
+        raise PkvError(1, "block_mapping must be [M, 2]")
+    _lib.check(_lib.load().copy_blocks(
+        ctypes.byref(desc), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_mapping, "block_mapping", torch.int32), int(block_mapping.shape[0]),
+        _dev(err_flag, "err_flag", torch.int32), _stream(stream)))
+
+
+def paged_attention_partition_size(k_cache, num_seqs: int, num_heads: int,
+                                   max_blocks_per_seq: int) -> int:
+    desc = cache_desc(k_cache)
+    return int(_lib.load().paged_attention_partition_size(ctypes.byref(desc), num_seqs, num_heads,
+                                                          max_blocks_per_seq))
+
+
+def paged_attention_workspace_bytes(k_cache, num_seqs: int, num_heads: int,
+                                    max_blocks_per_seq: int, partition_size: int = 0) -> int:
+    desc = cache_desc(k_cache)
+    return int(_lib.load().paged_attention_workspace_bytes(
+        ctypes.byref(desc), num_seqs, num_heads, max_blocks_per_seq, partition_size))
+
+
+def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                           partition_size: int = 0, workspace=None, err_flag=None, stream=None):
+    """out[b, h] = softmax(scale * q[b, h] . K) V over context_lens[b] tokens read through
+    block_tables[b] (int32 [B, MB]).  `workspace` (uint8 CUDA tensor) is allocated with
+    torch when needed and not given.  Returns `out`."""
+    torch = _torch()
+    desc = cache_desc(k_cache)
+    B, H, D = q.shape
+    if tuple(out.shape) != (B, H, D) or out.dtype != q.dtype or q.dtype != k_cache.dtype:
+        raise PkvError(1, "q and out must be [B, H, D] of the cache dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise PkvError(1, "block_tables must be [B, MB] and context_lens [B]")
+    MB = int(block_tables.shape[1])
+    need = paged_attention_workspace_bytes(k_cache, B, H, MB, partition_size)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _lib.check(_lib.load().paged_attention_decode(
+        ctypes.byref(desc), _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"),
+        _dev(v_cache, "v_cache"), _dev(block_tables, "block_tables", torch.int32), MB,
+        _dev(context_lens, "context_lens", torch.int32), B, H, ctypes.c_float(scale),
+        int(partition_size), _dev(workspace, "workspace"), ws_bytes,
+        _dev(err_flag, "err_flag", torch.int32), _stream(stream)))
+    return out
+
+
+def launch_count() -> int:
+    """Kernels libpkv has launched in this process."""
+    return int(_lib.load().pkv_launch_count())
+
+
+class Pool:
+    """Host block manager (pkv_pool_* / pkv_seq_*): free pool, block tables,
+    reference counts, fork and copy on write.  Host memory only."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        lib = _lib.load()
+        self.num_blocks, self.block_size = int(num_blocks), int(block_size)
+        handle = ctypes.c_void_p()
+        order = None
+        if free_order is not None:
+            self._order = np.ascontiguousarray(free_order, dtype=np.int32)
+            order = self._order.ctypes.data_as(ctypes.c_void_p)
+        _lib.check(lib.pkv_pool_create(num_blocks, block_size, order, ctypes.byref(handle)))
+        self._h = handle
+        self._lib = lib
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.pkv_pool_destroy(self._h)
+            self._h = None
+
+    __del__ = close
+
+    def new_seq(self) -> int:
+        sid = ctypes.c_int32()
+        _lib.check(self._lib.pkv_seq_new(self._h, ctypes.byref(sid)))
+        return sid.value
+
+    def fork(self, parent: int) -> int:
+        sid = ctypes.c_int32()
+        _lib.check(self._lib.pkv_seq_fork(self._h, parent, ctypes.byref(sid)))
+        return sid.value
+
+    def reserve(self, seq: int, n_tokens: int):
+        """(slots int64 array, [(src, dst)] copy pairs)."""
+        slots = np.empty(max(1, n_tokens), dtype=np.int64)
+        pair = np.empty(2, dtype=np.int32)
+        n = ctypes.c_int32()
+        _lib.check(self._lib.pkv_seq_reserve(self._h, seq, n_tokens,
+                                             slots.ctypes.data_as(ctypes.c_void_p),
+                                             pair.ctypes.data_as(ctypes.c_void_p), ctypes.byref(n)))
+        return slots[:n_tokens], ([(int(pair[0]), int(pair[1]))] if n.value else [])
+
+    def cow(self, seq: int, logical_block: int):
+        pair = np.empty(2, dtype=np.int32)
+        n = ctypes.c_int32()
+        _lib.check(self._lib.pkv_seq_cow(self._h, seq, logical_block,
+                                         pair.ctypes.data_as(ctypes.c_void_p), ctypes.byref(n)))
+        return (int(pair[0]), int(pair[1])) if n.value else None
+
+    def free_seq(self, seq: int) -> None:
+        _lib.check(self._lib.pkv_seq_free(self._h, seq))
+
+    def length(self, seq: int) -> int:
+        n = ctypes.c_int64()
+        _lib.check(self._lib.pkv_seq_len(self._h, seq, ctypes.byref(n)))
+        return n.value
+
+    def table(self, seq: int):
+        n = ctypes.c_int32()
+        _lib.check(self._lib.pkv_seq_block_table(self._h, seq, None, 0, ctypes.byref(n)))
+        row = np.empty(max(1, n.value), dtype=np.int32)
+        _lib.check(self._lib.pkv_seq_block_table(self._h, seq, row.ctypes.data_as(ctypes.c_void_p),
+                                                 n.value, ctypes.byref(n)))
+        return [int(x) for x in row[:n.value]]
+
+    def block_tables(self, seqs, max_blocks_per_seq: int, pad: int = -1):
+        """(int32 [len(seqs), max_blocks_per_seq] tables, int32 [len(seqs)] lengths)."""
+        ids = np.ascontiguousarray(seqs, dtype=np.int32)
+        tables = np.empty((len(ids), max_blocks_per_seq), dtype=np.int32)
+        lens = np.empty(len(ids), dtype=np.int32)
+        _lib.check(self._lib.pkv_pool_block_tables(
+            self._h, ids.ctypes.data_as(ctypes.c_void_p), len(ids),
+            tables.ctypes.data_as(ctypes.c_void_p), max_blocks_per_seq,
+            lens.ctypes.data_as(ctypes.c_void_p), pad))
+        return tables, lens
+
+    def refcount(self, block: int) -> int:
+        r = ctypes.c_int32()
+        _lib.check(self._lib.pkv_pool_refcount(self._h, block, ctypes.byref(r)))
+        return r.value
+
+    def free_list(self):
+        n = ctypes.c_int32()
+        _lib.check(self._lib.pkv_pool_free_list(self._h, None, 0, ctypes.byref(n)))
+        out = np.empty(max(1, n.value), dtype=np.int32)
+        _lib.check(self._lib.pkv_pool_free_list(self._h, out.ctypes.data_as(ctypes.c_void_p),
+                                                n.value, ctypes.byref(n)))
+        return [int(x) for x in out[:n.value]]
+
+    def stats(self) -> dict:
+        s = _lib.Stats()
+        _lib.check(self._lib.pkv_pool_stats(self._h, ctypes.byref(s)))
+        return {name: int(getattr(s, name)) for name, _ in _lib.Stats._fields_}

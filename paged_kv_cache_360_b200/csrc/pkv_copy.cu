@@ -1,0 +1,142 @@
+// pkv_copy.cu -- the two data-movement steps of a decode step: appending the new
+// token's keys and values through the slot mapping, and copying shared blocks
+// on write.  Both are pure HBM copies done with 16-byte vector loads and stores.
+//
+// "PagedAttention" ops page, How it works -- The mechanics: each decode step
+// writes the new token's key and value into the sequence's current block;
+// sequences that share blocks copy a block when they diverge.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pkv.h"
+#include "pkv_internal.h"
+
+namespace pkv {
+namespace {
+
+constexpr int kCopyThreads = 256;
+
+// One thread per 16-byte chunk of one (token, kv head) row, for K and V alike.
+// Consecutive threads cover consecutive chunks, so both the reads of `key` and
+// the writes into the pool are fully coalesced 128-bit accesses.
+__global__ void __launch_bounds__(kCopyThreads)
+append_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+              const uint4* __restrict__ key, const uint4* __restrict__ value,
+              const int64_t* __restrict__ slot_mapping, int64_t total_chunks,
+              int32_t chunks_per_row, int32_t num_kv_heads, int32_t block_size,
+              int64_t num_slots, int32_t* err_flag) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_chunks;
+         i += stride) {
+        const int64_t row = i / chunks_per_row;  // token * num_kv_heads + head
+        const int32_t c = static_cast<int32_t>(i - row * chunks_per_row);
+        const int64_t token = row / num_kv_heads;
+        const int32_t head = static_cast<int32_t>(row - token * num_kv_heads);
+        const int64_t slot = __ldg(slot_mapping + token);
+        if (slot < 0) continue;  // padding token
+        if (slot >= num_slots) {
+            if (c == 0 && head == 0 && err_flag) atomicOr(err_flag, PKV_DEVERR_BAD_SLOT);
+            continue;
+        }
+        const int64_t block = slot / block_size;
+        const int64_t offset = slot - block * block_size;
+        const int64_t dst = ((block * num_kv_heads + head) * block_size + offset) * chunks_per_row + c;
+        k_cache[dst] = __ldg(key + i);
+        v_cache[dst] = __ldg(value + i);
+    }
+}
+
+// grid = (pair, pool [0 = K, 1 = V], slice).  A block is contiguous in the pool
+// ([num_kv_heads][block_size][head_dim] elements), so each copy is one linear
+// run of `block_chunks` 16-byte chunks split over gridDim.z CTAs.
+__global__ void __launch_bounds__(kCopyThreads)
+copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                   const int32_t* __restrict__ block_mapping, int64_t block_chunks,
+                   int32_t num_blocks, int32_t* err_flag) {
+    const int32_t src = __ldg(block_mapping + 2 * blockIdx.x);
+    const int32_t dst = __ldg(block_mapping + 2 * blockIdx.x + 1);
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+        if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && err_flag)
+            atomicOr(err_flag, PKV_DEVERR_BAD_PAIR);
+        return;
+    }
+    uint4* pool = blockIdx.y == 0 ? k_cache : v_cache;
+    const uint4* from = pool + static_cast<int64_t>(src) * block_chunks;
+    uint4* to = pool + static_cast<int64_t>(dst) * block_chunks;
+    const int64_t stride = static_cast<int64_t>(gridDim.z) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.z) * blockDim.x + threadIdx.x; i < block_chunks;
+         i += stride)
+        to[i] = from[i];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+pkv_status check_desc(const pkv_cache_desc* d, const char* who) {
+    if (!d) return fail(PKV_ERR_INVALID_ARG, who);
+    if (d->num_blocks <= 0 || d->num_kv_heads <= 0 || d->block_size <= 0 || d->head_dim <= 0)
+        return fail(PKV_ERR_INVALID_ARG, "cache descriptor has a non-positive size");
+    if (d->dtype != PKV_F16 && d->dtype != PKV_BF16)
+        return fail(PKV_ERR_UNSUPPORTED, "dtype must be PKV_F16 or PKV_BF16");
+    if (d->head_dim != 64 && d->head_dim != 128)
+        return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+    if (d->block_size != 16 && d->block_size != 32)
+        return fail(PKV_ERR_UNSUPPORTED, "block_size must be 16 or 32");
+    return PKV_OK;
+}
+
+}  // namespace
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" pkv_status paged_kv_append(const pkv_cache_desc* desc, void* k_cache, void* v_cache,
+                                      const void* key, const void* value,
+                                      const int64_t* slot_mapping, int32_t num_tokens,
+                                      int32_t* err_flag, void* stream) {
+    pkv_status st = check_desc(desc, "paged_kv_append: desc is NULL");
+    if (st != PKV_OK) return st;
+    if (num_tokens < 0) return fail(PKV_ERR_INVALID_ARG, "paged_kv_append: num_tokens < 0");
+    if (num_tokens == 0) return PKV_OK;
+    if (!k_cache || !v_cache || !key || !value || !slot_mapping)
+        return fail(PKV_ERR_INVALID_ARG, "paged_kv_append: NULL pointer");
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(key) || !aligned16(value))
+        return fail(PKV_ERR_INVALID_ARG, "paged_kv_append: pools, key and value must be 16-byte aligned");
+    const int32_t chunks_per_row = desc->head_dim * 2 / 16;
+    const int64_t total = static_cast<int64_t>(num_tokens) * desc->num_kv_heads * chunks_per_row;
+    const int64_t want = (total + kCopyThreads - 1) / kCopyThreads;
+    const int grid = static_cast<int>(want < 148 * 16 ? want : 148 * 16);
+    append_kernel<<<grid, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<const uint4*>(key),
+        static_cast<const uint4*>(value), slot_mapping, total, chunks_per_row, desc->num_kv_heads,
+        desc->block_size, static_cast<int64_t>(desc->num_blocks) * desc->block_size, err_flag);
+    note_launches(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+    return PKV_OK;
+}
+
+extern "C" pkv_status copy_blocks(const pkv_cache_desc* desc, void* k_cache, void* v_cache,
+                                  const int32_t* block_mapping, int32_t num_pairs,
+                                  int32_t* err_flag, void* stream) {
+    pkv_status st = check_desc(desc, "copy_blocks: desc is NULL");
+    if (st != PKV_OK) return st;
+    if (num_pairs < 0) return fail(PKV_ERR_INVALID_ARG, "copy_blocks: num_pairs < 0");
+    if (num_pairs == 0) return PKV_OK;
+    if (!k_cache || !v_cache || !block_mapping)
+        return fail(PKV_ERR_INVALID_ARG, "copy_blocks: NULL pointer");
+    if (!aligned16(k_cache) || !aligned16(v_cache))
+        return fail(PKV_ERR_INVALID_ARG, "copy_blocks: pools must be 16-byte aligned");
+    const int64_t block_chunks =
+        static_cast<int64_t>(desc->num_kv_heads) * desc->block_size * desc->head_dim * 2 / 16;
+    // about 4 chunks (64 B) per thread per CTA
+    int64_t slices = (block_chunks + kCopyThreads * 4 - 1) / (kCopyThreads * 4);
+    if (slices > 65535) slices = 65535;
+    dim3 grid(static_cast<unsigned>(num_pairs), 2, static_cast<unsigned>(slices));
+    copy_blocks_kernel<<<grid, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), block_mapping, block_chunks,
+        desc->num_blocks, err_flag);
+    note_launches(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+    return PKV_OK;
+}

@@ -1,0 +1,258 @@
+// pkv_pool.cpp -- host block manager of the paged KV cache.
+//
+// Data structures of the "PagedAttention" ops page (Concept -- What it is; How it
+// works -- The mechanics) and the KV-cache lesson's analogy table: one pool of
+// fixed-size blocks, a free stack, a block table and length per sequence, and a
+// reference count per block.  Blocks are handed out one at a time when a
+// sequence's last block is full, go back to the free stack when their count
+// drops to zero, and a block that other sequences share is copied before a
+// sequence writes into it.  The tie-breaks (LIFO free stack seeded by a
+// caller-given order, logical-order release, ids counting up, all-or-nothing
+// requests) are stated in pkv.h.
+#include <cstdint>
+#include <new>
+#include <unordered_set>
+#include <vector>
+
+#include "pkv.h"
+#include "pkv_internal.h"
+
+struct pkv_pool {
+    int32_t num_blocks = 0;
+    int32_t block_size = 0;
+    std::vector<int32_t> free_stack;  // back() is the top
+    std::vector<int32_t> refcount;
+    struct Seq {
+        bool live = false;
+        int64_t len = 0;
+        std::vector<int32_t> blocks;
+    };
+    std::vector<Seq> seqs;  // index = sequence id
+
+    Seq* find(int32_t id) {
+        if (id < 0 || id >= static_cast<int32_t>(seqs.size()) || !seqs[id].live) return nullptr;
+        return &seqs[id];
+    }
+    const Seq* find(int32_t id) const {
+        if (id < 0 || id >= static_cast<int32_t>(seqs.size()) || !seqs[id].live) return nullptr;
+        return &seqs[id];
+    }
+    int32_t pop() {
+        int32_t b = free_stack.back();
+        free_stack.pop_back();
+        refcount[b] = 1;
+        return b;
+    }
+};
+
+using pkv::fail;
+
+extern "C" pkv_status pkv_pool_create(int32_t num_blocks, int32_t block_size,
+                                      const int32_t* free_order, pkv_pool** out) {
+    if (!out) return fail(PKV_ERR_INVALID_ARG, "pkv_pool_create: out is NULL");
+    *out = nullptr;
+    if (num_blocks <= 0 || block_size <= 0)
+        return fail(PKV_ERR_INVALID_ARG, "pkv_pool_create: num_blocks and block_size must be > 0");
+    pkv_pool* p = new (std::nothrow) pkv_pool();
+    if (!p) return fail(PKV_ERR_INVALID_ARG, "pkv_pool_create: out of host memory");
+    p->num_blocks = num_blocks;
+    p->block_size = block_size;
+    p->refcount.assign(num_blocks, 0);
+    p->free_stack.resize(num_blocks);
+    if (free_order) {
+        std::vector<char> seen(num_blocks, 0);
+        for (int32_t i = 0; i < num_blocks; ++i) {
+            int32_t b = free_order[i];
+            if (b < 0 || b >= num_blocks || seen[b]) {
+                delete p;
+                return fail(PKV_ERR_INVALID_ARG,
+                            "pkv_pool_create: free_order is not a permutation of the block ids");
+            }
+            seen[b] = 1;
+        }
+    }
+    // free_order[0] ends on top of the stack.
+    for (int32_t i = 0; i < num_blocks; ++i)
+        p->free_stack[num_blocks - 1 - i] = free_order ? free_order[i] : i;
+    *out = p;
+    return PKV_OK;
+}
+
+extern "C" void pkv_pool_destroy(pkv_pool* pool) { delete pool; }
+
+extern "C" pkv_status pkv_seq_new(pkv_pool* pool, int32_t* seq_id) {
+    if (!pool || !seq_id) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_new: NULL argument");
+    pool->seqs.emplace_back();
+    pool->seqs.back().live = true;
+    *seq_id = static_cast<int32_t>(pool->seqs.size() - 1);
+    return PKV_OK;
+}
+
+extern "C" pkv_status pkv_seq_fork(pkv_pool* pool, int32_t parent, int32_t* child) {
+    if (!pool || !child) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_fork: NULL argument");
+    if (!pool->find(parent)) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_fork: unknown parent");
+    pkv_pool::Seq copy = *pool->find(parent);
+    for (int32_t b : copy.blocks) pool->refcount[b] += 1;
+    pool->seqs.push_back(std::move(copy));
+    *child = static_cast<int32_t>(pool->seqs.size() - 1);
+    return PKV_OK;
+}
+
+extern "C" pkv_status pkv_seq_reserve(pkv_pool* pool, int32_t seq, int32_t n_tokens,
+                                      int64_t* slots_out, int32_t* cow_pair_out,
+                                      int32_t* n_cow_out) {
+    if (!pool || n_tokens < 0 || (n_tokens > 0 && !slots_out))
+        return fail(PKV_ERR_INVALID_ARG, "pkv_seq_reserve: bad argument");
+    pkv_pool::Seq* s = pool->find(seq);
+    if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_reserve: unknown sequence");
+    const int64_t bs = pool->block_size;
+    if (n_cow_out) *n_cow_out = 0;
+    // Blocks needed: one per block boundary crossed, plus a copy if the first
+    // token lands in a shared, partly filled block.
+    const int64_t have = (s->len + bs - 1) / bs;
+    const int64_t want = (s->len + n_tokens + bs - 1) / bs;
+    int64_t need = want - have;
+    const bool cow = n_tokens > 0 && s->len % bs != 0 &&
+                     pool->refcount[s->blocks[s->len / bs]] > 1;
+    if (cow) {
+        need += 1;
+        if (!cow_pair_out || !n_cow_out)
+            return fail(PKV_ERR_INVALID_ARG,
+                        "pkv_seq_reserve: the write needs a copy but cow_pair_out is NULL");
+    }
+    if (need > static_cast<int64_t>(pool->free_stack.size()))
+        return fail(PKV_ERR_NO_FREE_BLOCK, "pkv_seq_reserve: free pool exhausted");
+    if (cow) {
+        const int64_t i = s->len / bs;
+        const int32_t src = s->blocks[i];
+        const int32_t dst = pool->pop();
+        pool->refcount[src] -= 1;
+        s->blocks[i] = dst;
+        cow_pair_out[0] = src;
+        cow_pair_out[1] = dst;
+        *n_cow_out = 1;
+    }
+    for (int32_t k = 0; k < n_tokens; ++k) {
+        const int64_t pos = s->len;
+        if (pos % bs == 0) s->blocks.push_back(pool->pop());
+        slots_out[k] = static_cast<int64_t>(s->blocks[pos / bs]) * bs + pos % bs;
+        s->len = pos + 1;
+    }
+    return PKV_OK;
+}
+
+extern "C" pkv_status pkv_seq_cow(pkv_pool* pool, int32_t seq, int32_t logical_block,
+                                  int32_t* pair_out, int32_t* n_out) {
+    if (!pool || !pair_out || !n_out) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_cow: NULL argument");
+    pkv_pool::Seq* s = pool->find(seq);
+    if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_cow: unknown sequence");
+    if (logical_block < 0 || logical_block >= static_cast<int32_t>(s->blocks.size()))
+        return fail(PKV_ERR_INVALID_ARG, "pkv_seq_cow: logical block out of range");
+    *n_out = 0;
+    const int32_t src = s->blocks[logical_block];
+    if (pool->refcount[src] <= 1) return PKV_OK;
+    if (pool->free_stack.empty())
+        return fail(PKV_ERR_NO_FREE_BLOCK, "pkv_seq_cow: free pool exhausted");
+    const int32_t dst = pool->pop();
+    pool->refcount[src] -= 1;
+    s->blocks[logical_block] = dst;
+    pair_out[0] = src;
+    pair_out[1] = dst;
+    *n_out = 1;
+    return PKV_OK;
+}
+
+extern "C" pkv_status pkv_seq_free(pkv_pool* pool, int32_t seq) {
+    if (!pool) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_free: NULL pool");
+    pkv_pool::Seq* s = pool->find(seq);
+    if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_free: unknown sequence");
+    for (int32_t b : s->blocks) {
+        if (--pool->refcount[b] == 0) pool->free_stack.push_back(b);
+    }
+    s->blocks.clear();
+    s->blocks.shrink_to_fit();
+    s->len = 0;
+    s->live = false;
+    return PKV_OK;
+}
+
+extern "C" pkv_status pkv_seq_len(const pkv_pool* pool, int32_t seq, int64_t* len) {
+    if (!pool || !len) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_len: NULL argument");
+    const pkv_pool::Seq* s = pool->find(seq);
+    if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_len: unknown sequence");
+    *len = s->len;
+    return PKV_OK;
+}
+
+extern "C" pkv_status pkv_seq_block_table(const pkv_pool* pool, int32_t seq, int32_t* row,
+                                          int32_t cap, int32_t* n) {
+    if (!pool || !n || (cap > 0 && !row))
+        return fail(PKV_ERR_INVALID_ARG, "pkv_seq_block_table: bad argument");
+    const pkv_pool::Seq* s = pool->find(seq);
+    if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_block_table: unknown sequence");
+    *n = static_cast<int32_t>(s->blocks.size());
+    for (int32_t i = 0; i < *n && i < cap; ++i) row[i] = s->blocks[i];
+    return PKV_OK;
+}
+
+extern "C" pkv_status pkv_pool_block_tables(const pkv_pool* pool, const int32_t* seqs,
+                                            int32_t n_seqs, int32_t* tables,
+                                            int32_t max_blocks_per_seq, int32_t* context_lens,
+                                            int32_t pad) {
+    if (!pool || n_seqs < 0 || max_blocks_per_seq <= 0 ||
+        (n_seqs > 0 && (!seqs || !tables || !context_lens)))
+        return fail(PKV_ERR_INVALID_ARG, "pkv_pool_block_tables: bad argument");
+    for (int32_t i = 0; i < n_seqs; ++i) {
+        const pkv_pool::Seq* s = pool->find(seqs[i]);
+        if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_pool_block_tables: unknown sequence");
+        if (static_cast<int64_t>(s->blocks.size()) > max_blocks_per_seq)
+            return fail(PKV_ERR_INVALID_ARG,
+                        "pkv_pool_block_tables: a sequence has more blocks than max_blocks_per_seq");
+        if (s->len > INT32_MAX) return fail(PKV_ERR_INVALID_ARG, "pkv_pool_block_tables: length overflow");
+    }
+    for (int32_t i = 0; i < n_seqs; ++i) {
+        const pkv_pool::Seq* s = pool->find(seqs[i]);
+        int32_t* row = tables + static_cast<int64_t>(i) * max_blocks_per_seq;
+        const int32_t nb = static_cast<int32_t>(s->blocks.size());
+        for (int32_t j = 0; j < max_blocks_per_seq; ++j) row[j] = j < nb ? s->blocks[j] : pad;
+        context_lens[i] = static_cast<int32_t>(s->len);
+    }
+    return PKV_OK;
+}
+
+extern "C" pkv_status pkv_pool_refcount(const pkv_pool* pool, int32_t block, int32_t* refcount) {
+    if (!pool || !refcount || block < 0 || block >= pool->num_blocks)
+        return fail(PKV_ERR_INVALID_ARG, "pkv_pool_refcount: bad argument");
+    *refcount = pool->refcount[block];
+    return PKV_OK;
+}
+
+extern "C" pkv_status pkv_pool_free_list(const pkv_pool* pool, int32_t* out, int32_t cap,
+                                         int32_t* n) {
+    if (!pool || !n || (cap > 0 && !out))
+        return fail(PKV_ERR_INVALID_ARG, "pkv_pool_free_list: bad argument");
+    const int32_t total = static_cast<int32_t>(pool->free_stack.size());
+    *n = total;
+    for (int32_t i = 0; i < total && i < cap; ++i) out[i] = pool->free_stack[total - 1 - i];
+    return PKV_OK;
+}
+
+extern "C" pkv_status pkv_pool_stats(const pkv_pool* pool, pkv_stats* st) {
+    if (!pool || !st) return fail(PKV_ERR_INVALID_ARG, "pkv_pool_stats: NULL argument");
+    const int64_t bs = pool->block_size;
+    st->free_blocks = static_cast<int64_t>(pool->free_stack.size());
+    st->allocated_slots = (pool->num_blocks - st->free_blocks) * bs;
+    st->live_tokens = 0;
+    st->num_seqs = 0;
+    std::unordered_set<int64_t> live;
+    for (const auto& s : pool->seqs) {
+        if (!s.live) continue;
+        st->num_seqs += 1;
+        st->live_tokens += s.len;
+        for (int64_t t = 0; t < s.len; ++t) live.insert(static_cast<int64_t>(s.blocks[t / bs]) * bs + t % bs);
+    }
+    st->live_slots = static_cast<int64_t>(live.size());
+    st->shared_blocks = 0;
+    for (int32_t r : pool->refcount) st->shared_blocks += r > 1;
+    return PKV_OK;
+}

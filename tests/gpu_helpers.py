@@ -1,0 +1,66 @@
+"""Shared helpers of the GPU parity tests: move a workload to the device, run the
+library's calls, run the oracle on the same host buffers, compare."""
+
+import numpy as np
+import torch
+
+import oracle
+import paged_kv_cache_360_b200 as pkv
+from paged_kv_cache_360_b200 import _build
+
+# Per element: |gpu - oracle| <= ATOL + RTOL * |oracle|  (oracle in float64).
+ATOL = 2e-3
+RTOL = 1e-2
+
+
+def ensure_built():
+    _build.build()
+
+
+class Dev:
+    """A workload's buffers on cuda:0."""
+
+    def __init__(self, wl):
+        self.wl = wl
+        self.q = wl.q.cuda()
+        self.k = wl.k_cache.cuda()
+        self.v = wl.v_cache.cuda()
+        self.tables = torch.from_numpy(np.ascontiguousarray(wl.block_tables)).cuda()
+        self.lens = torch.from_numpy(np.ascontiguousarray(wl.context_lens)).cuda()
+        self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def decode(self, partition_size=0, tables=None, k=None, v=None):
+        out = torch.empty_like(self.q)
+        self.err.zero_()
+        pkv.paged_attention_decode(out, self.q, self.k if k is None else k,
+                                   self.v if v is None else v,
+                                   self.tables if tables is None else tables, self.lens,
+                                   self.wl.scale, partition_size=partition_size, err_flag=self.err)
+        torch.cuda.synchronize()
+        return out
+
+
+def oracle_decode(wl, seqs=None, k=None, v=None, tables=None):
+    return oracle.paged_decode(wl.q, wl.k_cache if k is None else k, wl.v_cache if v is None else v,
+                               wl.block_tables if tables is None else tables, wl.context_lens,
+                               wl.scale, seqs=seqs)
+
+
+def compare(gpu_out, ref, seqs=None, what=""):
+    g = gpu_out.detach().float().cpu().double().numpy()
+    if seqs is not None:
+        g, ref = g[seqs], ref[seqs]
+    err = np.abs(g - ref)
+    bound = ATOL + RTOL * np.abs(ref)
+    bad = ~(err <= bound)
+    if bad.any():
+        idx = np.argwhere(bad)[:5]
+        raise AssertionError(
+            f"{what}: {int(bad.sum())} of {bad.size} elements outside {ATOL} + {RTOL}|ref|; "
+            f"max abs {err.max():.3e}, first {idx.tolist()} gpu {g[bad][:5]} ref {ref[bad][:5]}")
+    rel = err / np.maximum(np.abs(ref), 1e-30)
+    return float(err.max()), float(np.where(np.abs(ref) > 1e-3, rel, 0).max())
+
+
+def words(t):
+    return oracle.words(t)

@@ -1,0 +1,105 @@
+"""The library's C++ block manager against the oracle's model, bit for bit (no GPU):
+the hand-traced golden traces, and long seeded random operation sequences with
+tables, slots, copy pairs, reference counts, free lists and statistics compared
+after every step."""
+
+import numpy as np
+import pytest
+
+from oracle.bookkeeping import BlockPoolModel, PoolExhausted as ModelExhausted
+from paged_kv_cache_360_b200 import Pool, PoolExhausted
+from tests.trace_player import play
+
+
+def _lib_pool(nb, bs, order):
+    return Pool(nb, bs, order)
+
+
+@pytest.mark.parametrize("trace", ["bookkeeping_trace.txt", "pool_exhaustion.txt"])
+def test_golden_traces_on_the_library(trace):
+    assert play(trace, _lib_pool, PoolExhausted) > 10
+
+
+def _same(model, pool, live):
+    assert pool.free_list() == model.free_list()
+    assert pool.stats() == {k: v for k, v in model.stats().items()} | {}
+    for sid in live:
+        assert pool.table(sid) == model.table(sid)
+        assert pool.length(sid) == model.length(sid)
+    for b in range(model.num_blocks):
+        assert pool.refcount(b) == model.refcount[b]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_operation_sequences_match_the_model(seed):
+    rng = np.random.default_rng(100 + seed)
+    nb, bs = int(rng.integers(8, 64)), int(rng.choice([1, 2, 4, 16]))
+    order = rng.permutation(nb)
+    model, pool = BlockPoolModel(nb, bs, order), Pool(nb, bs, order)
+    live = []
+    for step in range(500):
+        r = rng.random()
+        if r < 0.12 or not live:
+            a, b = model.new_seq(), pool.new_seq()
+            assert a == b
+            live.append(a)
+        elif r < 0.22:
+            parent = int(rng.choice(live))
+            a, b = model.fork(parent), pool.fork(parent)
+            assert a == b
+            live.append(a)
+        elif r < 0.75:
+            sid, n = int(rng.choice(live)), int(rng.integers(0, 2 * bs + 2))
+            try:
+                ms, mp = model.reserve(sid, n)
+            except ModelExhausted:
+                with pytest.raises(PoolExhausted):
+                    pool.reserve(sid, n)
+            else:
+                ls, lp = pool.reserve(sid, n)
+                assert list(ls) == ms and lp == [tuple(p) for p in mp]
+        elif r < 0.82:
+            sid = int(rng.choice(live))
+            nblk = len(model.table(sid))
+            if nblk:
+                i = int(rng.integers(0, nblk))
+                try:
+                    mp = model.cow(sid, i)
+                except ModelExhausted:
+                    with pytest.raises(PoolExhausted):
+                        pool.cow(sid, i)
+                else:
+                    assert pool.cow(sid, i) == mp
+        else:
+            sid = int(rng.choice(live))
+            live.remove(sid)
+            model.free_seq(sid)
+            pool.free_seq(sid)
+        _same(model, pool, live)
+
+
+def test_decode_step_export_matches_tables():
+    pool = Pool(32, 4, np.random.default_rng(0).permutation(32))
+    ids = [pool.new_seq() for _ in range(3)]
+    for sid, n in zip(ids, (5, 0, 9)):
+        pool.reserve(sid, n)
+    tables, lens = pool.block_tables(ids, 4, pad=-1)
+    for row, sid in zip(tables, ids):
+        t = pool.table(sid)
+        assert list(row[:len(t)]) == t and all(x == -1 for x in row[len(t):])
+    assert list(lens) == [5, 0, 9]
+
+
+def test_library_rejects_misuse():
+    from paged_kv_cache_360_b200 import PkvError
+    with pytest.raises(PkvError):
+        Pool(4, 2, [0, 0, 1, 2])                 # not a permutation
+    pool = Pool(4, 2)
+    with pytest.raises(PkvError):
+        pool.reserve(0, 1)                       # unknown sequence
+    sid = pool.new_seq()
+    pool.free_seq(sid)
+    with pytest.raises(PkvError):
+        pool.free_seq(sid)                       # already freed
+    with pytest.raises(PkvError):
+        pool.refcount(9)
