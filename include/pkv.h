@@ -162,6 +162,41 @@ pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* out, const v
                                   void* workspace, size_t workspace_bytes, int32_t* err_flag,
                                   void* stream);
 
+/*
+ * Decode without a caller workspace, for callers that cannot allocate device
+ * memory: a plugin inside a serving engine whose allocator already holds nearly
+ * all of the GPU's memory, or a latency-critical loop that must never call
+ * cudaMalloc (it synchronises the device and can fail when memory is
+ * fragmented).  The paper (the pages this library follows) has no
+ * counterpart to this call.
+ *
+ * Same arguments and result as paged_attention_decode without workspace /
+ * workspace_bytes: the partial results of split sequences go to a fixed
+ * PKV_STATIC_SCRATCH_BYTES array compiled into the library, which every GPU
+ * that loads the library holds until the process exits.  Shapes whose
+ * paged_attention_workspace_bytes(...) exceeds that size are rejected with
+ * PKV_ERR_WORKSPACE_TOO_SMALL and nothing is enqueued.  The call allocates
+ * nothing.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call on a device uses the same array, which keeps the last call's
+ *     contents; nothing in it needs to start at zero.  Calls that can run at the
+ *     same time on the GPU (different streams, no ordering) race on the array
+ *     and give wrong results: order them on one stream, or use
+ *     paged_attention_decode with separate workspaces.
+ */
+#define PKV_STATIC_SCRATCH_BYTES (16u << 20) /* 16 MiB */
+pkv_status paged_attention_decode_static_scratch(const pkv_cache_desc* desc, void* out,
+                                                 const void* q, const void* k_cache,
+                                                 const void* v_cache,
+                                                 const int32_t* block_tables,
+                                                 int32_t max_blocks_per_seq,
+                                                 const int32_t* context_lens, int32_t num_seqs,
+                                                 int32_t num_heads, float scale,
+                                                 int32_t partition_size, int32_t* err_flag,
+                                                 void* stream);
+
 /* -------------------------------------------------- host block bookkeeping */
 /*
  * The block manager of [ops page] Concept and How it works and the [lesson]

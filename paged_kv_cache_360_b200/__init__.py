@@ -20,8 +20,8 @@ from ._lib import PkvError, PoolExhausted  # noqa: F401
 
 __all__ = [
     "paged_kv_append", "copy_blocks", "paged_attention_decode", "paged_attention_workspace_bytes",
-    "paged_attention_partition_size", "Pool", "PkvError", "PoolExhausted", "launch_count",
-    "cache_desc",
+    "paged_attention_partition_size", "paged_attention_decode_static_scratch", "Pool",
+    "PkvError", "PoolExhausted", "launch_count", "cache_desc",
 ]
 
 
@@ -128,6 +128,29 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
         _dev(context_lens, "context_lens", torch.int32), B, H, ctypes.c_float(scale),
         int(partition_size), _dev(workspace, "workspace"), ws_bytes,
         _dev(err_flag, "err_flag", torch.int32), _stream(stream)))
+    return out
+
+
+def paged_attention_decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens,
+                                          scale, partition_size: int = 0, err_flag=None,
+                                          stream=None):
+    """paged_attention_decode for callers that cannot allocate device memory: the
+    split path uses the library's fixed 16 MiB scratch array instead of a
+    workspace (shapes needing more raise PkvError).  Calls that may run at the
+    same time on the GPU race on that array.  Returns `out`."""
+    torch = _torch()
+    desc = cache_desc(k_cache)
+    B, H, D = q.shape
+    if tuple(out.shape) != (B, H, D) or out.dtype != q.dtype or q.dtype != k_cache.dtype:
+        raise PkvError(1, "q and out must be [B, H, D] of the cache dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise PkvError(1, "block_tables must be [B, MB] and context_lens [B]")
+    _lib.check(_lib.load().paged_attention_decode_static_scratch(
+        ctypes.byref(desc), _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"),
+        _dev(v_cache, "v_cache"), _dev(block_tables, "block_tables", torch.int32),
+        int(block_tables.shape[1]), _dev(context_lens, "context_lens", torch.int32), B, H,
+        ctypes.c_float(scale), int(partition_size), _dev(err_flag, "err_flag", torch.int32),
+        _stream(stream)))
     return out
 
 

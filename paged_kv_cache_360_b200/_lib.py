@@ -20,11 +20,13 @@ DEVERR_BAD_CONTEXT_LEN = 2
 DEVERR_BAD_SLOT = 4
 DEVERR_WAIT_TIMEOUT = 8
 DEVERR_BAD_PAIR = 16
+STATIC_SCRATCH_BYTES = 16 << 20
 
 # Every function include/pkv.h declares (checked by the tests against the header).
 EXPORTS = (
     "paged_kv_append", "copy_blocks", "paged_attention_partition_size",
     "paged_attention_workspace_bytes", "paged_attention_decode",
+    "paged_attention_decode_static_scratch",
     "pkv_pool_create", "pkv_pool_destroy", "pkv_seq_new", "pkv_seq_fork", "pkv_seq_reserve",
     "pkv_seq_cow", "pkv_seq_free", "pkv_seq_len", "pkv_seq_block_table", "pkv_pool_block_tables",
     "pkv_pool_refcount", "pkv_pool_free_list", "pkv_pool_stats",
@@ -78,6 +80,8 @@ def load():
                 "paged_attention_workspace_bytes": (sz, [P(CacheDesc), i32, i32, i32, i32]),
                 "paged_attention_decode": (st, [P(CacheDesc), p, p, p, p, p, i32, p, i32, i32,
                                                 ctypes.c_float, i32, p, sz, p, p]),
+                "paged_attention_decode_static_scratch": (st, [P(CacheDesc), p, p, p, p, p, i32, p,
+                                                               i32, i32, ctypes.c_float, i32, p, p]),
                 "pkv_pool_create": (st, [i32, i32, p, P(p)]),
                 "pkv_pool_destroy": (None, [p]),
                 "pkv_seq_new": (st, [p, P(i32)]),

@@ -653,3 +653,71 @@ extern "C" pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* o
     if (desc->dtype == PKV_BF16) return dispatch_shape<__nv_bfloat16>(desc, tk, tv, a, num_seqs, split, s);
     return dispatch_shape<__half>(desc, tk, tv, a, num_seqs, split, s);
 }
+
+// ------------------------------------------------ decode without allocation
+//
+// Some callers cannot hand this library a workspace: a plugin running inside a
+// serving engine whose allocator has already reserved nearly all device memory
+// for its own pools, or a real-time decode loop that may not call cudaMalloc
+// (it synchronises the device and can fail under fragmentation).  For them,
+// paged_attention_decode_static_scratch keeps the split path's partial results
+// in a fixed array compiled into this file instead.
+namespace pkv {
+namespace {
+
+constexpr size_t kStaticScratchBytes = static_cast<size_t>(PKV_STATIC_SCRATCH_BYTES);
+
+// Every GPU that loads this library holds this array until the process exits.
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_scratch_addr[kMaxDevices];
+
+// Device address of g_static_scratch on the current device, looked up once
+// per device.  In host code the array's name is only a stand-in, never a
+// device address, so it must not be passed to a kernel directly.
+pkv_status static_scratch_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(PKV_ERR_UNSUPPORTED, "device index >= 64");
+    void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(PKV_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed");
+        g_scratch_addr[dev].store(p, std::memory_order_release);
+    }
+    *out = p;
+    return PKV_OK;
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" pkv_status paged_attention_decode_static_scratch(
+    const pkv_cache_desc* desc, void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+    int32_t num_seqs, int32_t num_heads, float scale, int32_t partition_size, int32_t* err_flag,
+    void* stream) {
+    pkv_status st = check_desc(desc);
+    if (st != PKV_OK) return st;
+    if (num_seqs < 0 || num_heads <= 0 || max_blocks_per_seq <= 0 || partition_size < 0)
+        return fail(PKV_ERR_INVALID_ARG,
+                    "paged_attention_decode_static_scratch: bad num_seqs, num_heads, "
+                    "max_blocks_per_seq or partition_size");
+    const size_t need = paged_attention_workspace_bytes(desc, num_seqs, num_heads,
+                                                        max_blocks_per_seq, partition_size);
+    if (need > kStaticScratchBytes)
+        return fail(PKV_ERR_WORKSPACE_TOO_SMALL,
+                    "paged_attention_decode_static_scratch: these shapes need more scratch than "
+                    "the 16 MiB static array holds (use paged_attention_decode with a workspace)");
+    void* scratch = nullptr;
+    if (need > 0 && (st = static_scratch_address(&scratch)) != PKV_OK) return st;
+    // No part of the scratch has to start at zero: every partial result the
+    // merge reads is written earlier in the same call.
+    return paged_attention_decode(desc, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                  context_lens, num_seqs, num_heads, scale, partition_size,
+                                  need > 0 ? scratch : nullptr, need > 0 ? kStaticScratchBytes : 0,
+                                  err_flag, stream);
+}
