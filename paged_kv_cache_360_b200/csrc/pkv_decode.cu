@@ -54,7 +54,11 @@ struct Geom {
     static constexpr int kHalfBytes = BS * 128;           // one half of one (block, head) tile
     static constexpr int kTileBytes = kHalves * kHalfBytes;  // K (or V) of one (block, head)
     static constexpr int kStageBytes = 2 * kTileBytes;    // K + V
-    static constexpr int kStages = kStageBytes <= 8192 ? 8 : 6;
+    // Stage s is always consumed by warp s % kConsumerWarps, so a warp waits on
+    // the rounds of its stages in order and is never a phase ahead of the
+    // barrier it polls (a parity wait cannot tell phase r-1 from phase r+1).
+    static constexpr int kStages = kStageBytes <= 8192 ? 8 : 4;
+    static_assert(kStages % kConsumerWarps == 0, "each stage must belong to one consumer warp");
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kMergeBytes = kConsumerWarps * 16 * (D + 2) * 4;
     static constexpr int kBodyBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
