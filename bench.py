@@ -224,7 +224,7 @@ def run_ours(args, rank, world, local_rank):
     d_lens = torch.from_numpy(lens).to(dev)
     out = torch.empty_like(q)
     B, H = wl.num_seqs, wl.num_heads
-    P = wl.partition_size or pkv.paged_attention_partition_size(k, B, H, tables.shape[1])
+    P = args.partition_size if args.partition_size is not None else wl.partition_size
     ws_bytes = pkv.paged_attention_workspace_bytes(k, B, H, tables.shape[1], P)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -345,7 +345,9 @@ def run_ours(args, rank, world, local_rank):
                    "num_heads": H, "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                    "block_size": wl.block_size, "num_blocks": wl.num_blocks,
                    "mean_context_len": float(np.mean(lens)), "max_context_len": int(np.max(lens)),
-                   "partition_size": int(P), "copy_pairs": int(len(pairs)),
+                   "partition_size": int(P),
+                   "schedule": "balanced" if P == 0 else f"fixed partitions of {P} tokens",
+                   "copy_pairs": int(len(pairs)),
                    "appended_tokens": int(len(slots)), "seed": args.seed,
                    "parallelism": f"dp{world} (independent batches per GPU)",
                    "l2": "not flushed: the step reads %.0f MB of K/V, %.1fx the 126 MB L2"
@@ -483,6 +485,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--partition-size", type=int, default=None,
+                    help="0 = balanced split (default unless the workload fixes one); "
+                         "> 0 = fixed partitions of that many tokens")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU time")

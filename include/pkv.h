@@ -109,19 +109,19 @@ pkv_status copy_blocks(const pkv_cache_desc* desc, void* k_cache, void* v_cache,
                        void* stream);
 
 /*
- * Partition size (tokens) the decode uses when called with partition_size 0:
- * 0 means "one pass per (sequence, kv head), no split"; otherwise a multiple of
- * block_size.  Depends only on the arguments and the current device's SM count.
- */
-int32_t paged_attention_partition_size(const pkv_cache_desc* desc, int32_t num_seqs,
-                                       int32_t num_heads, int32_t max_blocks_per_seq);
-
-/*
  * Workspace bytes paged_attention_decode needs for these shapes and
- * partition_size (0 = the library's choice above).  0 when no split is used.
- * Layout (float32): partial outputs [num_seqs][num_heads][P_max][head_dim], then
- * maxima and sums [num_seqs][num_heads][P_max] each, with
- * P_max = ceil(max_blocks_per_seq * block_size / partition_size).
+ * partition_size.
+ *   partition_size 0 (balanced): 2 * G * (group * (head_dim + 2) * 4 + 16) bytes,
+ *     G = resident CTAs of the decode on the current device (SM count x CTAs
+ *     per SM), group = num_heads / num_kv_heads.  Layout: partial outputs
+ *     float [G][2][group][head_dim], partial maxima and sums float
+ *     [G][2][group][2], partial descriptors int32 [G][2][4].
+ *   partition_size > 0 (fixed): 0 when partition_size >= max_blocks_per_seq *
+ *     block_size (no split); else float partial outputs
+ *     [num_seqs][num_heads][P_max][head_dim], then maxima and sums
+ *     [num_seqs][num_heads][P_max] each, P_max = ceil(max_blocks_per_seq *
+ *     block_size / partition_size).
+ * Returns 0 on invalid arguments.
  */
 size_t paged_attention_workspace_bytes(const pkv_cache_desc* desc, int32_t num_seqs,
                                        int32_t num_heads, int32_t max_blocks_per_seq,
@@ -146,9 +146,15 @@ size_t paged_attention_workspace_bytes(const pkv_cache_desc* desc, int32_t num_s
  *   block_tables    device int32 [num_seqs][max_blocks_per_seq]; entries at or
  *                   past ceil(context_len / block_size) are not read.
  *   context_lens    device int32 [num_seqs]; 0 gives an output of zeros.
- *   partition_size  0 = library's choice; otherwise a multiple of block_size;
- *                   sequences longer than it are split into partitions whose
- *                   partial results a second kernel merges by log-sum-exp.
+ *   partition_size  0 = balanced: the whole batch's work -- one unit per
+ *                   (sequence, kv head, block) -- is split evenly over the
+ *                   GPU's resident CTAs, whatever the length mix; sequences
+ *                   that straddle two CTAs are merged by a second kernel
+ *                   (log-sum-exp, in CTA order).  Results then depend on the
+ *                   device's SM count (not on timing).
+ *                   > 0 = fixed partitions of partition_size tokens (a multiple
+ *                   of block_size), merged by log-sum-exp in partition order;
+ *                   >= max_blocks_per_seq * block_size means no split.
  *   workspace       device, >= paged_attention_workspace_bytes(...), 16-byte
  *                   aligned; may be NULL when that size is 0.
  *   err_flag        device int32 or NULL (PKV_DEVERR_BAD_BLOCK_ID,

@@ -20,7 +20,7 @@ from ._lib import PkvError, PoolExhausted  # noqa: F401
 
 __all__ = [
     "paged_kv_append", "copy_blocks", "paged_attention_decode", "paged_attention_workspace_bytes",
-    "paged_attention_partition_size", "paged_attention_decode_static_scratch", "Pool",
+    "paged_attention_decode_static_scratch", "Pool",
     "PkvError", "PoolExhausted", "launch_count", "cache_desc",
 ]
 
@@ -91,13 +91,6 @@ def copy_blocks(k_cache, v_cache, block_mapping, err_flag=None, stream=None):
         _dev(err_flag, "err_flag", torch.int32), _stream(stream)))
 
 
-def paged_attention_partition_size(k_cache, num_seqs: int, num_heads: int,
-                                   max_blocks_per_seq: int) -> int:
-    desc = cache_desc(k_cache)
-    return int(_lib.load().paged_attention_partition_size(ctypes.byref(desc), num_seqs, num_heads,
-                                                          max_blocks_per_seq))
-
-
 def paged_attention_workspace_bytes(k_cache, num_seqs: int, num_heads: int,
                                     max_blocks_per_seq: int, partition_size: int = 0) -> int:
     desc = cache_desc(k_cache)
@@ -108,8 +101,10 @@ def paged_attention_workspace_bytes(k_cache, num_seqs: int, num_heads: int,
 def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale,
                            partition_size: int = 0, workspace=None, err_flag=None, stream=None):
     """out[b, h] = softmax(scale * q[b, h] . K) V over context_lens[b] tokens read through
-    block_tables[b] (int32 [B, MB]).  `workspace` (uint8 CUDA tensor) is allocated with
-    torch when needed and not given.  Returns `out`."""
+    block_tables[b] (int32 [B, MB]).  partition_size 0 splits the batch's work evenly
+    over the GPU (the default); > 0 uses fixed partitions of that many tokens.
+    `workspace` (uint8 CUDA tensor) is allocated with torch when needed and not
+    given.  Returns `out`."""
     torch = _torch()
     desc = cache_desc(k_cache)
     B, H, D = q.shape

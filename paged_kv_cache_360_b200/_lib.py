@@ -24,8 +24,7 @@ STATIC_SCRATCH_BYTES = 16 << 20
 
 # Every function include/pkv.h declares (checked by the tests against the header).
 EXPORTS = (
-    "paged_kv_append", "copy_blocks", "paged_attention_partition_size",
-    "paged_attention_workspace_bytes", "paged_attention_decode",
+    "paged_kv_append", "copy_blocks", "paged_attention_workspace_bytes", "paged_attention_decode",
     "paged_attention_decode_static_scratch",
     "pkv_pool_create", "pkv_pool_destroy", "pkv_seq_new", "pkv_seq_fork", "pkv_seq_reserve",
     "pkv_seq_cow", "pkv_seq_free", "pkv_seq_len", "pkv_seq_block_table", "pkv_pool_block_tables",
@@ -76,7 +75,6 @@ def load():
             sig = {
                 "paged_kv_append": (st, [P(CacheDesc), p, p, p, p, p, i32, p, p]),
                 "copy_blocks": (st, [P(CacheDesc), p, p, p, i32, p, p]),
-                "paged_attention_partition_size": (i32, [P(CacheDesc), i32, i32, i32]),
                 "paged_attention_workspace_bytes": (sz, [P(CacheDesc), i32, i32, i32, i32]),
                 "paged_attention_decode": (st, [P(CacheDesc), p, p, p, p, p, i32, p, i32, i32,
                                                 ctypes.c_float, i32, p, sz, p, p]),

@@ -6,29 +6,36 @@
 // What it is: a per-sequence block table maps logical positions to physical
 // blocks.
 //
-// Work item = (sequence b, kv head hk, partition p) = one CTA.  A partition is
-// `partition_tokens` consecutive logical tokens (a multiple of the block size),
-// or the whole sequence when the call does not split.
+// Both schedules below share one CTA shape -- 4 consumer warps + 1 producer warp
+// -- and the tile arithmetic of pkv_attend.cuh:
+//   * the producer issues, per logical block, TMA 2-D tiled loads of the (block,
+//     kv head) K and V tiles -- bs rows x 128 B per 64-column half, 128B swizzle
+//     -- into a ring of shared-memory stages, completion counted on one mbarrier
+//     per stage.  The tensor map spans the whole pool viewed as
+//     [num_blocks * num_kv_heads * bs rows][head_dim], so the gather through the
+//     block table is just the row coordinate (block * num_kv_heads + hk) * bs;
+//   * stage s belongs to consumer warp s % 4; all g = num_heads / num_kv_heads
+//     query heads of the kv head share each tile (S = Q K^T and O += P V on
+//     mma.sync m16n8k16, fp32 accumulate, online softmax in base 2);
+//   * the four warps' (m, l, O) are merged in shared memory in warp order.
 //
-// CTA = 4 consumer warps + 1 producer warp.
-//   * Producer: reads the partition's block-table entries (one coalesced load per
-//     32 blocks), and for each logical block issues TMA 2-D tiled loads of the
-//     (block, kv head) K and V tiles -- bs rows x 128 B per 64-column half, 128B
-//     swizzle -- into a ring of shared-memory stages, completion counted on an
-//     mbarrier per stage.  The tensor map spans the whole pool viewed as
-//     [num_blocks * num_kv_heads * bs rows][head_dim], so the gather is just the
-//     row coordinate (block * num_kv_heads + hk) * bs.
-//   * Consumers: warp w takes the partition's logical blocks w, w+4, w+8, ...
-//     All g = num_heads / num_kv_heads query heads of the kv head share each K/V
-//     tile: S = Q K^T and O += P V run on mma.sync m16n8k16 with the g query
-//     heads as the 16-row M side (rows >= g are zero), fp32 accumulators, and an
-//     online softmax in base 2 (scale * log2 e folded into the scores).
-//   * The four warps' (m, l, O) are merged in shared memory in warp order; the
-//     result is either the normalised output or, when split, the partition's
-//     un-normalised O with its max m and sum l.
-// The reduce kernel merges partitions p = 0, 1, ... in ascending order.  Every
-// reduction order depends only on logical token order, never on physical block
-// ids or timing, so results are bit-identical under block permutation.
+// Fixed partitions (partition_size > 0): one CTA per (sequence, kv head,
+// partition of partition_size tokens); a partition's un-normalised O and its
+// (m, l) go to the workspace and reduce_kernel merges partitions p = 0, 1, ...
+//
+// Balanced (partition_size == 0): a persistent grid of G CTAs (the resident
+// count).  The work is the list of units (sequence b, kv head hk, logical block)
+// in that order, U of them; CTA c takes units [c*U/G, (c+1)*U/G), so every CTA
+// streams the same number of blocks (+-1).  Its range is a run of segments (one
+// per (b, hk)); the producer walks it, publishing one descriptor per segment --
+// with the segment's query rows copied in by a bulk copy -- before the segment's
+// tiles.  A segment that covers a whole (b, hk) is written out directly; the at
+// most two that do not (the first and the last of the range) leave partials
+// that balanced_reduce_kernel chains across neighbouring CTAs in CTA order.
+//
+// Every reduction order depends only on logical token order and on the shapes,
+// never on physical block ids or timing, so results are bit-identical under any
+// permutation of physical blocks.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -38,6 +45,7 @@
 #include <mutex>
 
 #include "pkv.h"
+#include "pkv_attend.cuh"
 #include "pkv_internal.h"
 #include "pkv_ptx.cuh"
 
@@ -50,22 +58,45 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D, int BS>
 struct Geom {
-    static constexpr int kHalves = D / 64;                // 128-byte column halves per row
-    static constexpr int kHalfBytes = BS * 128;           // one half of one (block, head) tile
+    static constexpr int kHalves = D / 64;                   // 128-byte column halves per row
+    static constexpr int kHalfBytes = BS * 128;              // one half of one (block, head) tile
     static constexpr int kTileBytes = kHalves * kHalfBytes;  // K (or V) of one (block, head)
-    static constexpr int kStageBytes = 2 * kTileBytes;    // K + V
+    static constexpr int kStageBytes = 2 * kTileBytes;       // K + V
     // Stage s is always consumed by warp s % kConsumerWarps, so a warp waits on
     // the rounds of its stages in order and is never a phase ahead of the
     // barrier it polls (a parity wait cannot tell phase r-1 from phase r+1).
     static constexpr int kStages = kStageBytes <= 8192 ? 8 : 4;
     static_assert(kStages % kConsumerWarps == 0, "each stage must belong to one consumer warp");
     static constexpr int kRingBytes = kStages * kStageBytes;
-    static constexpr int kMergeBytes = kConsumerWarps * 16 * (D + 2) * 4;
-    static constexpr int kBodyBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
-    static constexpr int kBarOffset = kBodyBytes;
-    static constexpr int kSmemBytes = kBarOffset + 2 * kStages * 8 + 1024;  // + 1 KB alignment slack
     static_assert(kHalfBytes % 1024 == 0, "128B-swizzled tiles must start on 1 KB boundaries");
 };
+
+__device__ __forceinline__ void consumer_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
+
+__device__ __forceinline__ void flag(int32_t* err, int32_t bit) {
+    if (err) atomicOr(err, bit);
+}
+
+__device__ __forceinline__ int clamp_len(int L, int max_len) {
+    return L < 0 ? 0 : (L > max_len ? max_len : L);
+}
+
+// Issue the K and V tiles of (physical block, kv head) into one ring stage.
+template <int D, int BS>
+__device__ __forceinline__ void load_tile(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                          uint32_t stage_addr, uint32_t full_bar, int phys,
+                                          int num_kv_heads, int hk, uint64_t policy) {
+    using G = Geom<D, BS>;
+    mbar_arrive_expect_tx(full_bar, G::kStageBytes);
+    const int y = (phys * num_kv_heads + hk) * BS;
+    // one box = every 64-column half of BS rows (see encode_pool_map)
+    tma_load_3d(stage_addr, tm_k, 0, y, 0, full_bar, policy);
+    tma_load_3d(stage_addr + G::kTileBytes, tm_v, 0, y, 0, full_bar, policy);
+}
+
+// =================================================================== fixed partitions
 
 struct DecodeArgs {
     void* out;
@@ -86,36 +117,26 @@ struct DecodeArgs {
     float scale_log2;
 };
 
-__device__ __forceinline__ void consumer_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
-}
-
-__device__ __forceinline__ void flag(int32_t* err, int32_t bit) {
-    if (err) atomicOr(err, bit);
-}
-
-// Keep the 16-bit halves of `v` whose token index (t for the low half, t + 1
-// for the high half) is below `end`; zero the others.
-__device__ __forceinline__ uint32_t keep_valid(uint32_t v, int t, int end) {
-    if (t >= end) return 0u;
-    if (t + 1 >= end) return v & 0xffffu;
-    return v;
-}
-
-__device__ __forceinline__ int clamp_len(int L, int max_len) {
-    return L < 0 ? 0 : (L > max_len ? max_len : L);
-}
+template <int D, int BS>
+struct FixedLayout {
+    using G = Geom<D, BS>;
+    static constexpr int kMergeBytes = kConsumerWarps * 16 * (D + 2) * 4;
+    static constexpr int kBodyBytes = G::kRingBytes > kMergeBytes ? G::kRingBytes : kMergeBytes;
+    static constexpr int kBarOffset = kBodyBytes;
+    static constexpr int kSmemBytes = kBarOffset + 2 * G::kStages * 8 + 1024;  // + alignment slack
+};
 
 template <typename T, int D, int BS, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const DecodeArgs a) {
     using G = Geom<D, BS>;
+    using Lay = FixedLayout<D, BS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t base = smem_addr(smem);
-    const uint32_t bar_full = base + G::kBarOffset;          // kStages x 8 B
+    const uint32_t bar_full = base + Lay::kBarOffset;        // kStages x 8 B
     const uint32_t bar_empty = bar_full + 8 * G::kStages;    // kStages x 8 B
 
     const int warp = threadIdx.x >> 5;
@@ -175,16 +196,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                         flag(a.err_flag, PKV_DEVERR_WAIT_TIMEOUT);
                         ok = 0;
                     } else {
-                        const uint32_t full = bar_full + 8 * s;
-                        mbar_arrive_expect_tx(full, G::kStageBytes);
-                        const int y = (pj * a.num_kv_heads + hk) * BS;
-                        const uint32_t kdst = base + s * G::kStageBytes;
-                        const uint32_t vdst = kdst + G::kTileBytes;
-#pragma unroll
-                        for (int h = 0; h < G::kHalves; ++h) {
-                            tma_load_2d(kdst + h * G::kHalfBytes, &tm_k, 64 * h, y, full, policy);
-                            tma_load_2d(vdst + h * G::kHalfBytes, &tm_v, 64 * h, y, full, policy);
-                        }
+                        load_tile<D, BS>(&tm_k, &tm_v, base + s * G::kStageBytes, bar_full + 8 * s,
+                                         pj, a.num_kv_heads, hk, policy);
                     }
                 }
             }
@@ -194,33 +207,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     }
 
     // -------------------------------------------------------------- consumers
-    const int g = lane >> 2;   // fragment row (query head within the group)
-    const int t4 = lane & 3;   // fragment column pair
     const int group = a.group;
     const T* qbase = static_cast<const T*>(a.q) +
                      (static_cast<int64_t>(b) * a.num_heads + static_cast<int64_t>(hk) * group) * D;
-
-    // Q as the A operand of S = Q K^T, one 16x16 fragment per 16 columns of D.
     uint32_t qa[D / 16][4];
-    {
-        const bool lo_ok = g < group, hi_ok = g + 8 < group;
-        const uint32_t* qlo = reinterpret_cast<const uint32_t*>(qbase + g * D);
-        const uint32_t* qhi = reinterpret_cast<const uint32_t*>(qbase + (g + 8) * D);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-            qa[kk][0] = lo_ok ? __ldg(qlo + 8 * kk + t4) : 0u;
-            qa[kk][1] = hi_ok ? __ldg(qhi + 8 * kk + t4) : 0u;
-            qa[kk][2] = lo_ok ? __ldg(qlo + 8 * kk + 4 + t4) : 0u;
-            qa[kk][3] = hi_ok ? __ldg(qhi + 8 * kk + 4 + t4) : 0u;
-        }
-    }
+    load_q_fragments<T, D>(qa, qbase, group, lane);
 
-    float o[D / 8][4];
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-    float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
-    const float sl2 = a.scale_log2;
-
+    SoftmaxState<D> st;
+    st.reset();
     for (int it = warp; it < nblk; it += kConsumerWarps) {
         const int s = it % G::kStages;
         const int round = it / G::kStages;
@@ -230,151 +224,32 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             break;
         }
         const uint32_t kst = base + s * G::kStageBytes;
-        const uint32_t vst = kst + G::kTileBytes;
         const int tok_blk = (blk_begin + it) * BS;
 #pragma unroll
         for (int sub = 0; sub < BS / 16; ++sub) {
             const int tok0 = tok_blk + sub * 16;
             if (tok0 >= t_end) break;
-
-            // S (16 query rows x 16 tokens) = Q K^T
-            float sc[2][4];
-#pragma unroll
-            for (int i = 0; i < 2; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = 0.f;
-            {
-                const int mi = lane >> 3;
-                const int r = sub * 16 + (mi >> 1) * 8 + (lane & 7);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int chunk = 2 * kk + (mi & 1);
-                    const uint32_t addr = kst + (chunk >> 3) * G::kHalfBytes + r * 128 +
-                                          (((chunk & 7) ^ (r & 7)) << 4);
-                    uint32_t kb[4];
-                    ldsm_x4(addr, kb);
-                    Mma<T>::run(sc[0], qa[kk], kb[0], kb[1]);
-                    Mma<T>::run(sc[1], qa[kk], kb[2], kb[3]);
-                }
-            }
-
-            // scale into base 2, mask tokens past the partition, row maxima
-            float mx_lo = -INFINITY, mx_hi = -INFINITY;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const bool valid = tok0 + nt * 8 + 2 * t4 + j < t_end;
-                    sc[nt][j] = valid ? sc[nt][j] * sl2 : -INFINITY;
-                    sc[nt][2 + j] = valid ? sc[nt][2 + j] * sl2 : -INFINITY;
-                    mx_lo = fmaxf(mx_lo, sc[nt][j]);
-                    mx_hi = fmaxf(mx_hi, sc[nt][2 + j]);
-                }
-            }
-            mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
-            mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
-            mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
-            mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
-            const float mn_lo = fmaxf(m_lo, mx_lo);
-            const float mn_hi = fmaxf(m_hi, mx_hi);
-            if (__any_sync(0xffffffffu, mn_lo != m_lo || mn_hi != m_hi)) {
-                const float al = exp2_approx(m_lo - mn_lo);
-                const float ah = exp2_approx(m_hi - mn_hi);
-                l_lo *= al;
-                l_hi *= ah;
-#pragma unroll
-                for (int i = 0; i < D / 8; ++i) {
-                    o[i][0] *= al;
-                    o[i][1] *= al;
-                    o[i][2] *= ah;
-                    o[i][3] *= ah;
-                }
-            }
-            m_lo = mn_lo;
-            m_hi = mn_hi;
-
-            // P = 2^(S - m), rounded to T: the A operand of O += P V.  The row
-            // sums use the rounded values, so the weights that multiply V are
-            // exactly the ones that normalise.
-            uint32_t pa[4];
-            {
-                float r0, r1;
-                pa[0] = Pack<T>::two(exp2_approx(sc[0][0] - mn_lo), exp2_approx(sc[0][1] - mn_lo), r0, r1);
-                l_lo += r0 + r1;
-                pa[1] = Pack<T>::two(exp2_approx(sc[0][2] - mn_hi), exp2_approx(sc[0][3] - mn_hi), r0, r1);
-                l_hi += r0 + r1;
-                pa[2] = Pack<T>::two(exp2_approx(sc[1][0] - mn_lo), exp2_approx(sc[1][1] - mn_lo), r0, r1);
-                l_lo += r0 + r1;
-                pa[3] = Pack<T>::two(exp2_approx(sc[1][2] - mn_hi), exp2_approx(sc[1][3] - mn_hi), r0, r1);
-                l_hi += r0 + r1;
-            }
-
-            // O (16 rows x D) += P (16 x 16 tokens) V (16 tokens x D)
-            {
-                const bool partial = tok0 + 16 > t_end;
-                const int mi = lane >> 3;
-                const int r = sub * 16 + (mi & 1) * 8 + (lane & 7);
-                const int ta = tok0 + 2 * t4, tb = tok0 + 8 + 2 * t4;
-#pragma unroll
-                for (int nd = 0; nd < D / 16; ++nd) {
-                    const int chunk = 2 * nd + (mi >> 1);
-                    const uint32_t addr = vst + (chunk >> 3) * G::kHalfBytes + r * 128 +
-                                          (((chunk & 7) ^ (r & 7)) << 4);
-                    uint32_t vb[4];
-                    ldsm_x4_trans(addr, vb);
-                    if (partial) {
-                        // rows past the end may hold anything (even NaN): zero them
-                        vb[0] = keep_valid(vb[0], ta, t_end);
-                        vb[2] = keep_valid(vb[2], ta, t_end);
-                        vb[1] = keep_valid(vb[1], tb, t_end);
-                        vb[3] = keep_valid(vb[3], tb, t_end);
-                    }
-                    Mma<T>::run(o[2 * nd], pa, vb[0], vb[1]);
-                    Mma<T>::run(o[2 * nd + 1], pa, vb[2], vb[3]);
-                }
-            }
+            attend_16<T, D>(st, qa, kst, kst + G::kTileBytes, G::kHalfBytes, sub, tok0, t_end,
+                            a.scale_log2, lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_empty + 8 * s);
     }
 
     // ----------------------------------------------- merge the four warps
-    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
-    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
-    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
-    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
-
+    finish_row_sums(st);
     consumer_sync();  // every consumer is done with the ring: reuse it
-    float* mo = reinterpret_cast<float*>(smem);              // [warp][16][D]
-    float* mm = mo + kConsumerWarps * 16 * D;                // [warp][16]
-    float* ml = mm + kConsumerWarps * 16;                    // [warp][16]
-    if (t4 == 0) {
-        mm[warp * 16 + g] = m_lo;
-        mm[warp * 16 + g + 8] = m_hi;
-        ml[warp * 16 + g] = l_lo;
-        ml[warp * 16 + g + 8] = l_hi;
-    }
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-        const int col = i * 8 + 2 * t4;
-        *reinterpret_cast<float2*>(mo + (warp * 16 + g) * D + col) = make_float2(o[i][0], o[i][1]);
-        *reinterpret_cast<float2*>(mo + (warp * 16 + g + 8) * D + col) = make_float2(o[i][2], o[i][3]);
-    }
+    float* mo = reinterpret_cast<float*>(smem);              // [warp][group][D]
+    float* mm = mo + kConsumerWarps * 16 * D;                // [warp][group]
+    float* ml = mm + kConsumerWarps * 16;                    // [warp][group]
+    store_warp_state(st, mo, mm, ml, warp, group, lane);
     consumer_sync();
 
-    const int tid = threadIdx.x;  // 0 .. 127 (consumers only)
-    for (int idx = tid; idx < group * D; idx += kConsumerWarps * 32) {
+    for (int idx = threadIdx.x; idx < group * D; idx += kConsumerWarps * 32) {
         const int r = idx / D;
         const int d = idx - r * D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mm[w * 16 + r]);
-        float acc = 0.f, den = 0.f;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-            const float mw = mm[w * 16 + r];
-            const float f = mw == -INFINITY ? 0.f : exp2_approx(mw - M);
-            acc += f * mo[(w * 16 + r) * D + d];
-            den += f * ml[w * 16 + r];
-        }
+        float M, acc, den;
+        combine_warps<D>(mo, mm, ml, kConsumerWarps, group, r, d, M, acc, den);
         const int64_t bh = static_cast<int64_t>(b) * a.num_heads + static_cast<int64_t>(hk) * group + r;
         if (SPLIT) {
             const int64_t slot = bh * a.max_partitions + part;
@@ -413,6 +288,552 @@ __global__ void __launch_bounds__(D) reduce_kernel(const DecodeArgs a, int32_t m
     static_cast<T*>(a.out)[bh * D + d] = Pack<T>::one(den > 0.f ? acc / den : 0.f);
 }
 
+// =========================================================================== balanced
+
+constexpr int kSegSlots = 4;          // segment descriptors in flight
+constexpr int kMergeSlots = 2;        // segments handed to the merge warp, in flight
+constexpr int kBalancedThreads = (kConsumerWarps + 2) * 32;  // + producer + merge warp
+constexpr int kMetaValid = 1;         // partial-slot meta flags
+constexpr int kMetaBegins = 2;        // the segment starts at the (b, hk)'s first block
+constexpr int kMetaEnds = 4;          // the segment ends at the (b, hk)'s last block
+constexpr int kSegFirstInCta = 8;     // descriptor-only flags
+constexpr int kSegEnd = 16;           // end of the CTA's range
+
+struct BalancedArgs {
+    void* out;
+    const void* q;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    float* ws_o;      // [G][2][group][D]   un-normalised partial O
+    float* ws_ml;     // [G][2][group][2]   partial (m, l)
+    int32_t* ws_meta; // [G][2][4]          (b, hk, flags, 0)
+    int32_t* err_flag;
+    int32_t num_seqs;
+    int32_t num_heads;
+    int32_t num_kv_heads;
+    int32_t group;
+    int32_t max_blocks_per_seq;
+    int32_t num_blocks;
+    float scale_log2;
+};
+
+struct SegDesc {
+    int32_t b, hk, first, n;  // CTA-local index of the first unit, unit count
+    int32_t blk0, len, flags, pad;
+};
+
+// The balanced kernel streams 16-token units: a block of 32 tokens is two units
+// (two TMA boxes of 16 rows), so every block size gets the same 64 KiB ring of
+// 8 KiB (head_dim 128) or 4 KiB (head_dim 64) stages, at least two per warp.
+template <int D>
+struct UnitGeom {
+    static constexpr int kHalves = D / 64;
+    static constexpr int kHalfBytes = 16 * 128;               // 16 rows x 128 B, 128B swizzle
+    static constexpr int kTileBytes = kHalves * kHalfBytes;
+    static constexpr int kStageBytes = 2 * kTileBytes;        // K + V
+    static constexpr int kRingBytes = 64 * 1024;
+    static constexpr int kStages = kRingBytes / kStageBytes;  // 8 or 16
+    static_assert(kStages % kConsumerWarps == 0, "each stage must belong to one consumer warp");
+};
+
+// Byte offsets inside the (1 KB aligned) dynamic shared memory of the balanced
+// kernel; the part after the ring depends on the group size.
+template <int D>
+struct BalancedLayout {
+    using G = UnitGeom<D>;
+    // merge slot: mo [warps][group][D], mm [warps][group], ml [warps][group], 4 ints
+    int qslot_bytes, q_off, mslot_bytes, merge_off, desc_off, bar_off, abort_off, total;
+    __host__ __device__ explicit BalancedLayout(int group) {
+        qslot_bytes = group * D * 2;                                   // multiple of 128
+        q_off = G::kRingBytes;
+        mslot_bytes = ((kConsumerWarps * group * (D + 2) * 4 + 16) + 15) & ~15;
+        merge_off = q_off + kSegSlots * qslot_bytes;
+        desc_off = merge_off + kMergeSlots * mslot_bytes;
+        bar_off = desc_off + kSegSlots * static_cast<int>(sizeof(SegDesc));
+        // full[S], empty[S], seg_full[4], seg_empty[4], mslot_full[2], mslot_empty[2]
+        abort_off = bar_off + (2 * G::kStages + 2 * kSegSlots + 2 * kMergeSlots) * 8;
+        total = abort_off + 16 + 1024;  // + 1 KB alignment slack
+    }
+};
+
+// Poll a barrier until the phase with `parity` completes, the limit runs out or
+// another warp has aborted; false unless the phase completed.
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
+                                              const volatile int* abort_word) {
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        if (mbar_test(bar, parity)) return true;
+        if ((i & 63) == 63 && *abort_word) return false;
+    }
+    return false;
+}
+
+// Issue the K and V tiles of one 16-token unit: rows [row0, row0 + 16) of the
+// pools' 2-D view.
+template <int D>
+__device__ __forceinline__ void load_unit(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                          uint32_t stage_addr, uint32_t full_bar, int row0,
+                                          uint64_t policy) {
+    using G = UnitGeom<D>;
+    mbar_arrive_expect_tx(full_bar, G::kStageBytes);
+    tma_load_3d(stage_addr, tm_k, 0, row0, 0, full_bar, policy);
+    tma_load_3d(stage_addr + G::kTileBytes, tm_v, 0, row0, 0, full_bar, policy);
+}
+
+// Up to 32 consecutive units of one (b, hk), with the physical block of each
+// unit held by lane j of the producer warp (unit j of the chunk).
+struct Chunk {
+    int b, hk, u0, cnt;   // sequence, kv head, first unit within (b, hk), units
+    int len, nu;          // the sequence's length and its units per kv head
+    int seg_start;        // the chunk opens a segment of seg_len units
+    int seg_len;
+    int phys;             // this lane's physical block
+};
+
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(kBalancedThreads, 2)
+balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                const BalancedArgs a) {
+    using G = UnitGeom<D>;
+    constexpr int R = BS / 16;  // units per block
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ long long s_warp_units[kConsumerWarps + 2];
+    __shared__ int s_start[3];
+
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int group = a.group;
+    const BalancedLayout<D> lay(group);
+    const uint32_t base = smem_addr(smem);
+    const uint32_t bar_full = base + lay.bar_off;
+    const uint32_t bar_empty = bar_full + 8 * G::kStages;
+    const uint32_t seg_full = bar_empty + 8 * G::kStages;
+    const uint32_t seg_empty = seg_full + 8 * kSegSlots;
+    const uint32_t mslot_full = seg_empty + 8 * kSegSlots;
+    const uint32_t mslot_empty = mslot_full + 8 * kMergeSlots;
+    volatile int* abort_word = reinterpret_cast<volatile int*>(smem + lay.abort_off);
+    SegDesc* descs = reinterpret_cast<SegDesc*>(smem + lay.desc_off);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int c = blockIdx.x;
+    const int grid = gridDim.x;
+    const int B = a.num_seqs;
+    const int Hkv = a.num_kv_heads;
+    const int max_len = a.max_blocks_per_seq * BS;
+
+    pdl_launch_dependents();
+    if (tid < 8) a.ws_meta[static_cast<int64_t>(c) * 8 + tid] = 0;  // both partial slots invalid
+
+    // ---- which units are this CTA's: units per sequence, scanned over the batch
+    const int chunk = (B + kBalancedThreads - 1) / kBalancedThreads;
+    const int b_lo = min(B, tid * chunk), b_hi = min(B, b_lo + chunk);
+    long long mine = 0;
+    for (int b = b_lo; b < b_hi; ++b) {
+        const int raw = __ldg(a.context_lens + b);
+        const int L = clamp_len(raw, max_len);
+        if (raw != L && c == 0) flag(a.err_flag, PKV_DEVERR_BAD_CONTEXT_LEN);
+        mine += (L + 15) / 16;
+    }
+    long long incl = mine;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    if (lane == 31) s_warp_units[warp] = incl;
+    if (tid == 0) s_start[0] = -1;
+    __syncthreads();
+    long long before = 0, total = 0;
+    for (int w = 0; w < kConsumerWarps + 2; ++w) {
+        if (w < warp) before += s_warp_units[w];
+        total += s_warp_units[w];
+    }
+    const long long excl = before + incl - mine;          // units (per kv head) before b_lo
+    const long long units = total * Hkv;
+    // Spread the units over min(G, U) CTAs, so that every range is non-empty and
+    // the CTAs that share one (b, hk) are consecutive.
+    const long long used = units < grid ? units : grid;
+    const long long u0 = c < used ? static_cast<long long>(c) * units / used : 0;
+    const long long u1 = c < used ? static_cast<long long>(c + 1) * units / used : 0;
+    if (u0 < u1 && mine > 0 && excl * Hkv <= u0 && u0 < (excl + mine) * Hkv) {
+        long long p = excl;
+        for (int b = b_lo; b < b_hi; ++b) {
+            const int nu = (clamp_len(__ldg(a.context_lens + b), max_len) + 15) / 16;
+            if (u0 < (p + nu) * Hkv) {
+                const long long r = u0 - p * Hkv;
+                s_start[0] = b;
+                s_start[1] = static_cast<int>(r / nu);
+                s_start[2] = static_cast<int>(r % nu);
+                break;
+            }
+            p += nu;
+        }
+    }
+    if (tid == 0) {
+        for (int s = 0; s < G::kStages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int k = 0; k < kSegSlots; ++k) {
+            mbar_init(seg_full + 8 * k, 1);
+            mbar_init(seg_empty + 8 * k, kConsumerWarps);
+        }
+        for (int k = 0; k < kMergeSlots; ++k) {
+            mbar_init(mslot_full + 8 * k, kConsumerWarps);
+            mbar_init(mslot_empty + 8 * k, 1);
+        }
+        *abort_word = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (u0 >= u1 || s_start[0] < 0) return;  // no units for this CTA
+    const int n_units = static_cast<int>(u1 - u0);
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------------ producer
+        // Walks the range chunk by chunk; the table entries (and the length of
+        // the next sequence) are loaded one chunk ahead, before the warp blocks
+        // on the ring, so a segment boundary costs no idle DRAM time.
+        if (lane == 0) {
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+        }
+        const uint64_t policy = l2_evict_first_policy();
+        int b = s_start[0], hk = s_start[1], ub = s_start[2];  // walk cursor
+        int len = clamp_len(__ldg(a.context_lens + b), max_len);
+        int nu = (len + 15) / 16;
+        // raw, clamped only when used, so the load does not stall the warp here
+        int len_next_raw = b + 1 < B ? __ldg(a.context_lens + b + 1) : 0;
+        int walked = 0;  // units already assigned to chunks
+
+        // Take the next chunk from the cursor and issue its table loads.
+        auto take = [&](Chunk& ch) -> bool {
+            if (ub == nu) {  // the (b, hk) is done: next kv head, or next sequence with tokens
+                ub = 0;
+                if (++hk == Hkv) {
+                    hk = 0;
+                    ++b;
+                    len = clamp_len(len_next_raw, max_len);
+                    while (len == 0 && b + 1 < B) {
+                        ++b;
+                        len = clamp_len(__ldg(a.context_lens + b), max_len);
+                    }
+                    nu = (len + 15) / 16;
+                    len_next_raw = b + 1 < B ? __ldg(a.context_lens + b + 1) : 0;
+                }
+            }
+            ch.b = b;
+            ch.hk = hk;
+            ch.u0 = ub;
+            ch.len = len;
+            ch.nu = nu;
+            ch.cnt = min(32, min(nu - ub, n_units - walked));
+            if (ch.cnt <= 0) return false;  // lengths changed under the kernel
+            ch.seg_start = ub == 0 || walked == 0;
+            ch.seg_len = min(nu - ub, n_units - walked);
+            // the entries are checked when they are used, so the loads stay in flight
+            ch.phys = lane < ch.cnt
+                          ? __ldg(a.block_tables + static_cast<int64_t>(b) * a.max_blocks_per_seq +
+                                  (ub + lane) / R)
+                          : 0;
+            ub += ch.cnt;
+            walked += ch.cnt;
+            return true;
+        };
+
+        int ok = 1, i = 0, seg = 0;
+        int tiles_issued = 0, queries_issued = 0;  // lane 0's counts of copies issued
+        Chunk cur, nxt;
+        ok = take(cur);
+        while (ok) {
+            const bool more = walked < n_units;
+            if (more && !take(nxt)) ok = 0;
+            if (!ok) break;
+            if (cur.seg_start) {
+                const int ks = seg % kSegSlots;
+                if (lane == 0) {
+                    if (seg >= kSegSlots &&
+                        !wait_or_abort(seg_empty + 8 * ks, ((seg / kSegSlots) - 1) & 1, abort_word)) {
+                        ok = 0;
+                    } else {
+                        SegDesc& d = descs[ks];
+                        d.b = cur.b;
+                        d.hk = cur.hk;
+                        d.first = i;
+                        d.n = cur.seg_len;
+                        d.blk0 = cur.u0;
+                        d.len = cur.len;
+                        d.flags = (cur.u0 == 0 ? kMetaBegins : 0) |
+                                  (cur.u0 + cur.seg_len == cur.nu ? kMetaEnds : 0) |
+                                  (i == 0 ? kSegFirstInCta : 0);
+                        // the arrive releases the descriptor's stores to the consumers
+                        mbar_arrive_expect_tx(seg_full + 8 * ks, lay.qslot_bytes);
+                        const T* qsrc = static_cast<const T*>(a.q) +
+                                        (static_cast<int64_t>(cur.b) * a.num_heads +
+                                         static_cast<int64_t>(cur.hk) * group) * D;
+                        bulk_load(base + lay.q_off + ks * lay.qslot_bytes, qsrc, lay.qslot_bytes,
+                                  seg_full + 8 * ks);
+                        ++queries_issued;
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                ++seg;
+                if (!ok) break;
+            }
+            for (int j = 0; j < cur.cnt; ++j) {
+                int pj = __shfl_sync(0xffffffffu, cur.phys, j);
+                if (pj < 0 || pj >= a.num_blocks) {
+                    if (lane == 0) flag(a.err_flag, PKV_DEVERR_BAD_BLOCK_ID);
+                    pj = 0;
+                }
+                if (lane == 0 && ok) {
+                    const int u = i + j;
+                    const int s = u % G::kStages;
+                    const int round = u / G::kStages;
+                    if (round > 0 && !wait_or_abort(bar_empty + 8 * s, (round - 1) & 1, abort_word)) {
+                        ok = 0;
+                    } else {
+                        const int row0 = (pj * Hkv + cur.hk) * BS + ((cur.u0 + j) % R) * 16;
+                        load_unit<D>(&tm_k, &tm_v, base + s * G::kStageBytes, bar_full + 8 * s, row0, policy);
+                        ++tiles_issued;
+                    }
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            i += cur.cnt;
+            if (!more || !ok) break;
+            cur = nxt;
+        }
+        if (lane == 0) {
+            if (ok) {
+                const int ks = seg % kSegSlots;
+                if (seg >= kSegSlots &&
+                    !wait_or_abort(seg_empty + 8 * ks, ((seg / kSegSlots) - 1) & 1, abort_word)) {
+                    ok = 0;
+                } else {
+                    descs[ks].n = 0;
+                    descs[ks].flags = kSegEnd;
+                    mbar_arrive(seg_full + 8 * ks);
+                }
+            }
+            if (!ok) {
+                // Timed out or aborted: flag it, and before leaving wait (bounded)
+                // for the copies this warp issued, so none lands after the CTA ends.
+                flag(a.err_flag, PKV_DEVERR_WAIT_TIMEOUT);
+                *abort_word = 1;
+                for (int s = 0; s < G::kStages && s < tiles_issued; ++s)
+                    mbar_wait(bar_full + 8 * s, ((tiles_issued - 1 - s) / G::kStages) & 1);
+                for (int k = 0; k < kSegSlots && k < queries_issued; ++k)
+                    mbar_wait(seg_full + 8 * k, ((queries_issued - 1 - k) / kSegSlots) & 1);
+            }
+        }
+        return;
+    }
+
+    if (warp == kConsumerWarps + 1) {
+        // ---------------------------------------------------------- merge warp
+        // Combines the four consumer warps' states of each segment, in segment
+        // order, while the consumers already work on the next one.
+        for (int seg = 0;; ++seg) {
+            const int ms = seg % kMergeSlots;
+            if (!__all_sync(0xffffffffu, wait_or_abort(mslot_full + 8 * ms, (seg / kMergeSlots) & 1, abort_word))) {
+                if (lane == 0) flag(a.err_flag, PKV_DEVERR_WAIT_TIMEOUT);
+                *abort_word = 1;
+                break;
+            }
+            const float* mo = reinterpret_cast<const float*>(smem + lay.merge_off + ms * lay.mslot_bytes);
+            const float* mm = mo + kConsumerWarps * group * D;
+            const float* ml = mm + kConsumerWarps * group;
+            const int* smeta = reinterpret_cast<const int*>(ml + kConsumerWarps * group);
+            const int flags = smeta[2];
+            if (flags & kSegEnd) break;
+            const int sb = smeta[0], shk = smeta[1];
+            const bool complete = (flags & (kMetaBegins | kMetaEnds)) == (kMetaBegins | kMetaEnds);
+            const int64_t pslot = static_cast<int64_t>(c) * 2 + ((flags & kSegFirstInCta) ? 0 : 1);
+            // Row by row: the weights 2^(m_w - M) once per row, then four columns
+            // per lane (M = max_w m_w; acc = sum_w 2^(m_w - M) o_w; den likewise).
+            for (int r = 0; r < group; ++r) {
+                float mw[kConsumerWarps], M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    mw[w] = mm[w * group + r];
+                    M = fmaxf(M, mw[w]);
+                }
+                float f[kConsumerWarps], den = 0.f;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    f[w] = mw[w] == -INFINITY ? 0.f : exp2_approx(mw[w] - M);
+                    den += f[w] * ml[w * group + r];
+                }
+                const int d0 = lane * 4;
+                if (d0 < D) {
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w) {
+                        const float4 o = *reinterpret_cast<const float4*>(mo + (w * group + r) * D + d0);
+                        acc.x += f[w] * o.x;
+                        acc.y += f[w] * o.y;
+                        acc.z += f[w] * o.z;
+                        acc.w += f[w] * o.w;
+                    }
+                    if (complete) {
+                        const float inv = den > 0.f ? 1.f / den : 0.f;
+                        float r0, r1;
+                        uint2 packed;
+                        packed.x = Pack<T>::two(acc.x * inv, acc.y * inv, r0, r1);
+                        packed.y = Pack<T>::two(acc.z * inv, acc.w * inv, r0, r1);
+                        const int64_t bh = static_cast<int64_t>(sb) * a.num_heads + static_cast<int64_t>(shk) * group + r;
+                        *reinterpret_cast<uint2*>(static_cast<T*>(a.out) + bh * D + d0) = packed;
+                    } else {
+                        *reinterpret_cast<float4*>(a.ws_o + (pslot * group + r) * D + d0) = acc;
+                        if (lane == 0) {
+                            a.ws_ml[(pslot * group + r) * 2] = M;
+                            a.ws_ml[(pslot * group + r) * 2 + 1] = den;
+                        }
+                    }
+                }
+            }
+            if (!complete && lane == 0) {
+                int32_t* meta = a.ws_meta + pslot * 4;
+                meta[0] = sb;
+                meta[1] = shk;
+                meta[2] = kMetaValid | (flags & (kMetaBegins | kMetaEnds));
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(mslot_empty + 8 * ms);  // the slot may be refilled
+        }
+        return;
+    }
+
+    // -------------------------------------------------------------- consumers
+    // Hand this warp's state of segment `seg` (or, with flags = kSegEnd, the end
+    // of the range) to the merge warp through merge slot seg % 2.
+    auto publish = [&](int seg, const SoftmaxState<D>& state, int b_, int hk_, int flags_) -> bool {
+        const int ms = seg % kMergeSlots;
+        if (seg >= kMergeSlots &&
+            !__all_sync(0xffffffffu,
+                        wait_or_abort(mslot_empty + 8 * ms, ((seg / kMergeSlots) - 1) & 1, abort_word)))
+            return false;
+        float* mo = reinterpret_cast<float*>(smem + lay.merge_off + ms * lay.mslot_bytes);
+        float* mm = mo + kConsumerWarps * group * D;
+        float* ml = mm + kConsumerWarps * group;
+        int* smeta = reinterpret_cast<int*>(ml + kConsumerWarps * group);
+        if (!(flags_ & kSegEnd)) store_warp_state(state, mo, mm, ml, warp, group, lane);
+        if (warp == 0 && lane == 0) {
+            smeta[0] = b_;
+            smeta[1] = hk_;
+            smeta[2] = flags_;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(mslot_full + 8 * ms);
+        return true;
+    };
+    SoftmaxState<D> st;
+    uint32_t qa[D / 16][4];
+    bool ok = true;
+    for (int seg = 0; ok; ++seg) {
+        const int ks = seg % kSegSlots;
+        if (!__all_sync(0xffffffffu, wait_or_abort(seg_full + 8 * ks, (seg / kSegSlots) & 1, abort_word))) {
+            ok = false;
+            break;
+        }
+        const SegDesc d = descs[ks];
+        if (d.flags & kSegEnd) {
+            ok = publish(seg, st, 0, 0, kSegEnd);  // the merge warp stops here
+            break;
+        }
+        load_q_fragments<T, D>(qa, reinterpret_cast<const T*>(smem + lay.q_off + ks * lay.qslot_bytes),
+                               group, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(seg_empty + 8 * ks);  // descriptor and queries are in registers
+
+        st.reset();
+        for (int u = d.first + ((warp - d.first) & 3); u < d.first + d.n; u += kConsumerWarps) {
+            const int s = u % G::kStages;
+            const int round = u / G::kStages;
+            if (!__all_sync(0xffffffffu, wait_or_abort(bar_full + 8 * s, round & 1, abort_word))) {
+                ok = false;
+                break;
+            }
+            const uint32_t kst = base + s * G::kStageBytes;
+            attend_16<T, D>(st, qa, kst, kst + G::kTileBytes, G::kHalfBytes, 0,
+                            (d.blk0 + (u - d.first)) * 16, d.len, a.scale_log2, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+        }
+        if (!ok) break;
+
+        finish_row_sums(st);
+        if (!publish(seg, st, d.b, d.hk, d.flags)) {
+            ok = false;
+            break;
+        }
+    }
+    if (!ok) {
+        if (lane == 0) flag(a.err_flag, PKV_DEVERR_WAIT_TIMEOUT);
+        *abort_word = 1;
+    }
+}
+
+// Merge the partials of every (b, hk) that was split across CTAs.  CTA c owns
+// the chains that start in it (a partial marked "begins"); a chain continues in
+// slot 0 of CTAs c+1, c+2, ... until a partial marked "ends".  Sequences with
+// no tokens get zeros here.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) balanced_reduce_kernel(const BalancedArgs a) {
+    pdl_wait_primary();
+    const int c = blockIdx.x;
+    const int grid = gridDim.x;
+    const int group = a.group;
+    for (int slot = 0; slot < 2; ++slot) {
+        const int32_t* meta = a.ws_meta + (static_cast<int64_t>(c) * 2 + slot) * 4;
+        const int flags = meta[2];
+        if (!(flags & kMetaValid) || !(flags & kMetaBegins)) continue;
+        const int b = meta[0], hk = meta[1];
+        for (int idx = threadIdx.x; idx < group * D; idx += blockDim.x) {
+            const int r = idx / D;
+            const int d = idx - r * D;
+            // the chain's length: up to and including the partial marked "ends"
+            int last = c;
+            bool broken = false;
+            if (!(flags & kMetaEnds)) {
+                for (;;) {
+                    ++last;
+                    const int32_t* nm = a.ws_meta + static_cast<int64_t>(last) * 8;
+                    if (last >= grid || !(nm[2] & kMetaValid) || nm[0] != b || nm[1] != hk) {
+                        broken = true;
+                        --last;
+                        break;
+                    }
+                    if (nm[2] & kMetaEnds) break;
+                }
+            }
+            if (broken && d == 0 && r == 0) flag(a.err_flag, PKV_DEVERR_WAIT_TIMEOUT);
+            float M = -INFINITY;
+            for (int cc = c; cc <= last; ++cc) {
+                const int64_t p = static_cast<int64_t>(cc) * 2 + (cc == c ? slot : 0);
+                M = fmaxf(M, a.ws_ml[(p * group + r) * 2]);
+            }
+            float acc = 0.f, den = 0.f;
+            for (int cc = c; cc <= last; ++cc) {
+                const int64_t p = static_cast<int64_t>(cc) * 2 + (cc == c ? slot : 0);
+                const float f = exp2_approx(a.ws_ml[(p * group + r) * 2] - M);
+                acc += f * a.ws_o[(p * group + r) * D + d];
+                den += f * a.ws_ml[(p * group + r) * 2 + 1];
+            }
+            const int64_t bh = static_cast<int64_t>(b) * a.num_heads + static_cast<int64_t>(hk) * group + r;
+            static_cast<T*>(a.out)[bh * D + d] = Pack<T>::one(den > 0.f ? acc / den : 0.f);
+        }
+    }
+    // sequences with no tokens: zeros (context lengths <= 0 count as empty)
+    for (int b = c; b < a.num_seqs; b += grid) {
+        if (__ldg(a.context_lens + b) > 0) continue;
+        T* o = static_cast<T*>(a.out) + static_cast<int64_t>(b) * a.num_heads * D;
+        for (int idx = threadIdx.x; idx < a.num_heads * D; idx += blockDim.x) o[idx] = Pack<T>::one(0.f);
+    }
+}
+
 // ------------------------------------------------------------------ host side
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -429,31 +850,28 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// A 2-D view of one pool: rows = num_blocks * num_kv_heads * block_size,
-// columns = head_dim; box = 64 columns (128 B) x block_size rows, 128B swizzle.
-pkv_status encode_pool_map(CUtensorMap* tm, const void* pool, const pkv_cache_desc* d) {
+// A 3-D view of one pool: x = 64 columns (128 B), y = row (num_blocks *
+// num_kv_heads * block_size rows of head_dim elements), z = which 64-column
+// half of the row (strides: 2 * head_dim bytes for y, 128 bytes for z).  A box
+// of 64 x box_rows x head_dim/64 lands in shared memory as [half][row][128 B],
+// 128B-swizzled, so one request fetches a whole (block, kv head) tile.
+pkv_status encode_pool_map(CUtensorMap* tm, const void* pool, const pkv_cache_desc* d, int box_rows) {
     auto encode = tensor_map_encoder();
     if (!encode) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     const cuuint64_t rows = static_cast<cuuint64_t>(d->num_blocks) * d->num_kv_heads * d->block_size;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(d->head_dim), rows};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(d->head_dim) * 2};
-    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(d->block_size)};
-    cuuint32_t estr[2] = {1, 1};
+    const cuuint32_t halves = static_cast<cuuint32_t>(d->head_dim / 64);
+    cuuint64_t dims[3] = {64, rows, halves};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d->head_dim) * 2, 128};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), halves};
+    cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = encode(tm,
                         d->dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                        2, const_cast<void*>(pool), dims, strides, box, estr,
+                        3, const_cast<void*>(pool), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     return PKV_OK;
-}
-
-int sm_count() {
-    int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess) return n;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
-    return n;
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -473,59 +891,45 @@ pkv_status check_desc(const pkv_cache_desc* d) {
     return PKV_OK;
 }
 
-// Library choice of partition size; 0 = no split.
-int32_t choose_partition(const pkv_cache_desc* d, int32_t num_seqs, int32_t max_blocks_per_seq) {
-    const int64_t max_len = static_cast<int64_t>(max_blocks_per_seq) * d->block_size;
-    int32_t P = 512;
-    if (max_len <= P) return 0;
-    const int64_t target = 4LL * sm_count();  // two resident CTAs per SM, two waves
-    const int64_t pairs = static_cast<int64_t>(num_seqs) * d->num_kv_heads;
-    while (P > 128 && pairs * ((max_len + P - 1) / P) < target) P /= 2;
-    if (P % d->block_size != 0) P = (P / d->block_size) * d->block_size;
-    return P;
-}
-
-int32_t resolve_partition(const pkv_cache_desc* d, int32_t num_seqs, int32_t max_blocks_per_seq,
-                          int32_t requested) {
-    const int64_t max_len = static_cast<int64_t>(max_blocks_per_seq) * d->block_size;
-    const int32_t P = requested == 0 ? choose_partition(d, num_seqs, max_blocks_per_seq) : requested;
-    return (P == 0 || P >= max_len) ? 0 : P;
-}
-
-size_t workspace_for(const pkv_cache_desc* d, int32_t num_seqs, int32_t num_heads,
-                     int32_t max_blocks_per_seq, int32_t P) {
-    if (P == 0) return 0;
-    const int64_t max_len = static_cast<int64_t>(max_blocks_per_seq) * d->block_size;
-    const int64_t pmax = (max_len + P - 1) / P;
-    return static_cast<size_t>(num_seqs) * num_heads * pmax * (d->head_dim + 2) * sizeof(float);
-}
-
-// Opt the kernel in to its dynamic shared memory once per device (the static
-// is per template instantiation, i.e. per kernel).
-template <typename T, int D, int BS, bool SPLIT>
-cudaError_t allow_smem() {
+// Opt a kernel in to the device's maximum dynamic shared memory, once per device
+// (the static is per template instantiation of K, and K is per kernel below).
+template <typename Tag>
+cudaError_t opt_in_smem(const void* kernel) {
     static std::atomic<uint64_t> done{0};
     int dev = 0;
-    cudaGetDevice(&dev);
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
     const uint64_t bit = 1ull << (dev & 63);
     if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D, BS, SPLIT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Geom<D, BS>::kSmemBytes);
+    int limit = 0;
+    if ((e = cudaDeviceGetAttribute(&limit, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+        return e;
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, kernel)) != cudaSuccess) return e;
+    // dynamic + static shared memory may not exceed the opt-in limit
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             limit - static_cast<int>(fa.sharedSizeBytes));
     if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_release);
     return e;
 }
 
+template <typename T, int D, int BS, bool SPLIT>
+struct FixedTag {};
 template <typename T, int D, int BS>
-pkv_status launch(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a,
-                  int32_t num_seqs, bool split, cudaStream_t stream) {
-    using G = Geom<D, BS>;
+struct BalancedTag {};
+
+template <typename T, int D, int BS>
+pkv_status launch_fixed(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a,
+                        int32_t num_seqs, bool split, cudaStream_t stream) {
+    using Lay = FixedLayout<D, BS>;
     const dim3 grid(static_cast<unsigned>(num_seqs) * a.num_kv_heads,
                     split ? static_cast<unsigned>(a.max_partitions) : 1u);
     cudaError_t e;
     if (split) {
-        if ((e = allow_smem<T, D, BS, true>()) != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
-        decode_kernel<T, D, BS, true><<<grid, kThreads, G::kSmemBytes, stream>>>(tk, tv, a);
+        auto k = decode_kernel<T, D, BS, true>;
+        if ((e = opt_in_smem<FixedTag<T, D, BS, true>>(reinterpret_cast<const void*>(k))) != cudaSuccess)
+            return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+        k<<<grid, kThreads, Lay::kSmemBytes, stream>>>(tk, tv, a);
         note_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
         // The merge launches as a programmatic dependent of the partition
@@ -534,7 +938,6 @@ pkv_status launch(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(num_seqs) * a.num_heads);
         cfg.blockDim = dim3(D);
-        cfg.dynamicSmemBytes = 0;
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -546,21 +949,103 @@ pkv_status launch(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs
         note_launches(1);
         if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
     } else {
-        if ((e = allow_smem<T, D, BS, false>()) != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
-        decode_kernel<T, D, BS, false><<<grid, kThreads, G::kSmemBytes, stream>>>(tk, tv, a);
+        auto k = decode_kernel<T, D, BS, false>;
+        if ((e = opt_in_smem<FixedTag<T, D, BS, false>>(reinterpret_cast<const void*>(k))) != cudaSuccess)
+            return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+        k<<<grid, kThreads, Lay::kSmemBytes, stream>>>(tk, tv, a);
         note_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
     }
     return PKV_OK;
 }
 
-template <typename T>
-pkv_status dispatch_shape(const pkv_cache_desc* d, const CUtensorMap& tk, const CUtensorMap& tv,
-                          const DecodeArgs& a, int32_t num_seqs, bool split, cudaStream_t st) {
-    if (d->head_dim == 128 && d->block_size == 16) return launch<T, 128, 16>(tk, tv, a, num_seqs, split, st);
-    if (d->head_dim == 128 && d->block_size == 32) return launch<T, 128, 32>(tk, tv, a, num_seqs, split, st);
-    if (d->head_dim == 64 && d->block_size == 16) return launch<T, 64, 16>(tk, tv, a, num_seqs, split, st);
-    return launch<T, 64, 32>(tk, tv, a, num_seqs, split, st);
+// Resident CTAs of the balanced kernel on the current device: its grid size.
+template <typename T, int D, int BS>
+pkv_status balanced_grid(int group, int* grid_out, int* smem_out) {
+    const BalancedLayout<D> lay(group);
+    auto k = balanced_kernel<T, D, BS>;
+    cudaError_t e = opt_in_smem<BalancedTag<T, D, BS>>(reinterpret_cast<const void*>(k));
+    if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kBalancedThreads, lay.total)) != cudaSuccess)
+        return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+    if (per_sm < 1) return fail(PKV_ERR_UNSUPPORTED, "balanced decode does not fit on an SM");
+    *grid_out = sms * per_sm;
+    *smem_out = lay.total;
+    return PKV_OK;
+}
+
+template <typename T, int D, int BS>
+pkv_status launch_balanced(const CUtensorMap& tk, const CUtensorMap& tv, const BalancedArgs& a,
+                           int grid, int smem, cudaStream_t stream) {
+    balanced_kernel<T, D, BS><<<grid, kBalancedThreads, smem, stream>>>(tk, tv, a);
+    note_launches(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, balanced_reduce_kernel<T, D>, a);
+    note_launches(1);
+    if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+    return PKV_OK;
+}
+
+// Dispatch on (dtype, head_dim, block_size) to F<T, D, BS>::run.
+template <template <typename, int, int> class F, typename... Args>
+pkv_status dispatch(const pkv_cache_desc* d, Args&&... args) {
+    if (d->dtype == PKV_BF16) {
+        if (d->head_dim == 128 && d->block_size == 16) return F<__nv_bfloat16, 128, 16>::run(args...);
+        if (d->head_dim == 128 && d->block_size == 32) return F<__nv_bfloat16, 128, 32>::run(args...);
+        if (d->head_dim == 64 && d->block_size == 16) return F<__nv_bfloat16, 64, 16>::run(args...);
+        return F<__nv_bfloat16, 64, 32>::run(args...);
+    }
+    if (d->head_dim == 128 && d->block_size == 16) return F<__half, 128, 16>::run(args...);
+    if (d->head_dim == 128 && d->block_size == 32) return F<__half, 128, 32>::run(args...);
+    if (d->head_dim == 64 && d->block_size == 16) return F<__half, 64, 16>::run(args...);
+    return F<__half, 64, 32>::run(args...);
+}
+
+template <typename T, int D, int BS>
+struct GridOf {
+    static pkv_status run(int group, int* grid, int* smem) { return balanced_grid<T, D, BS>(group, grid, smem); }
+};
+template <typename T, int D, int BS>
+struct RunFixed {
+    static pkv_status run(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a,
+                          int32_t num_seqs, bool split, cudaStream_t st) {
+        return launch_fixed<T, D, BS>(tk, tv, a, num_seqs, split, st);
+    }
+};
+template <typename T, int D, int BS>
+struct RunBalanced {
+    static pkv_status run(const CUtensorMap& tk, const CUtensorMap& tv, const BalancedArgs& a,
+                          int grid, int smem, cudaStream_t st) {
+        return launch_balanced<T, D, BS>(tk, tv, a, grid, smem, st);
+    }
+};
+
+// Workspace of the fixed-partition path (0 when it does not split).
+size_t fixed_workspace(const pkv_cache_desc* d, int32_t num_seqs, int32_t num_heads,
+                       int32_t max_blocks_per_seq, int32_t P) {
+    const int64_t max_len = static_cast<int64_t>(max_blocks_per_seq) * d->block_size;
+    if (P == 0 || P >= max_len) return 0;
+    const int64_t pmax = (max_len + P - 1) / P;
+    return static_cast<size_t>(num_seqs) * num_heads * pmax * (d->head_dim + 2) * sizeof(float);
+}
+
+// Workspace of the balanced path: two partial slots per CTA.
+size_t balanced_workspace(int grid, int group, int D) {
+    return static_cast<size_t>(grid) * 2 *
+           (static_cast<size_t>(group) * (D + 2) * sizeof(float) + 4 * sizeof(int32_t));
 }
 
 }  // namespace
@@ -568,21 +1053,19 @@ pkv_status dispatch_shape(const pkv_cache_desc* d, const CUtensorMap& tk, const 
 
 using namespace pkv;
 
-extern "C" int32_t paged_attention_partition_size(const pkv_cache_desc* desc, int32_t num_seqs,
-                                                  int32_t num_heads, int32_t max_blocks_per_seq) {
-    (void)num_heads;
-    if (check_desc(desc) != PKV_OK || num_seqs <= 0 || max_blocks_per_seq <= 0) return 0;
-    return resolve_partition(desc, num_seqs, max_blocks_per_seq, 0);
-}
-
 extern "C" size_t paged_attention_workspace_bytes(const pkv_cache_desc* desc, int32_t num_seqs,
                                                   int32_t num_heads, int32_t max_blocks_per_seq,
                                                   int32_t partition_size) {
     if (check_desc(desc) != PKV_OK || num_seqs <= 0 || num_heads <= 0 || max_blocks_per_seq <= 0 ||
-        partition_size < 0)
+        partition_size < 0 || num_heads % desc->num_kv_heads != 0)
         return 0;
-    const int32_t P = resolve_partition(desc, num_seqs, max_blocks_per_seq, partition_size);
-    return workspace_for(desc, num_seqs, num_heads, max_blocks_per_seq, P);
+    if (partition_size > 0)
+        return fixed_workspace(desc, num_seqs, num_heads, max_blocks_per_seq, partition_size);
+    const int group = num_heads / desc->num_kv_heads;
+    if (group > 16) return 0;
+    int grid = 0, smem = 0;
+    if (dispatch<GridOf>(desc, group, &grid, &smem) != PKV_OK) return 0;
+    return balanced_workspace(grid, group, desc->head_dim);
 }
 
 extern "C" pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* out, const void* q,
@@ -597,12 +1080,14 @@ extern "C" pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* o
     pkv_status st = check_desc(desc);
     if (st != PKV_OK) return st;
     if (num_seqs < 0 || num_heads <= 0 || max_blocks_per_seq <= 0)
-        return fail(PKV_ERR_INVALID_ARG, "paged_attention_decode: bad num_seqs, num_heads or max_blocks_per_seq");
+        return fail(PKV_ERR_INVALID_ARG,
+                    "paged_attention_decode: bad num_seqs, num_heads or max_blocks_per_seq");
     if (num_seqs == 0) return PKV_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
         return fail(PKV_ERR_INVALID_ARG, "paged_attention_decode: NULL pointer");
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
-        return fail(PKV_ERR_INVALID_ARG, "paged_attention_decode: q, out and pools must be 16-byte aligned");
+        return fail(PKV_ERR_INVALID_ARG,
+                    "paged_attention_decode: q, out and pools must be 16-byte aligned");
     if (num_heads % desc->num_kv_heads != 0)
         return fail(PKV_ERR_INVALID_ARG, "num_heads must be a multiple of num_kv_heads");
     const int32_t group = num_heads / desc->num_kv_heads;
@@ -611,14 +1096,47 @@ extern "C" pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* o
         return fail(PKV_ERR_INVALID_ARG, "scale must be finite");
     if (static_cast<int64_t>(max_blocks_per_seq) * desc->block_size > INT32_MAX / 2)
         return fail(PKV_ERR_UNSUPPORTED, "max_blocks_per_seq * block_size too large");
-    if (static_cast<int64_t>(num_seqs) * desc->num_kv_heads > INT32_MAX)
-        return fail(PKV_ERR_UNSUPPORTED, "num_seqs * num_kv_heads too large");
+    if (static_cast<int64_t>(num_seqs) * max_blocks_per_seq * desc->num_kv_heads > INT32_MAX)
+        return fail(PKV_ERR_UNSUPPORTED,
+                    "num_seqs * max_blocks_per_seq * num_kv_heads must be < 2^31");
     if (partition_size < 0 || (partition_size > 0 && partition_size % desc->block_size != 0))
-        return fail(PKV_ERR_INVALID_ARG, "partition_size must be 0 or a positive multiple of block_size");
+        return fail(PKV_ERR_INVALID_ARG,
+                    "partition_size must be 0 or a positive multiple of block_size");
 
-    const int32_t P = resolve_partition(desc, num_seqs, max_blocks_per_seq, partition_size);
-    const bool split = P != 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    CUtensorMap tk, tv;
+
+    if (partition_size == 0) {
+        int grid = 0, smem = 0;
+        if ((st = dispatch<GridOf>(desc, static_cast<int>(group), &grid, &smem)) != PKV_OK) return st;
+        const size_t need = balanced_workspace(grid, group, desc->head_dim);
+        if (!workspace || workspace_bytes < need)
+            return fail(PKV_ERR_WORKSPACE_TOO_SMALL, "paged_attention_decode: workspace too small");
+        if (!aligned(workspace, 16))
+            return fail(PKV_ERR_INVALID_ARG, "paged_attention_decode: workspace must be 16-byte aligned");
+        if ((st = encode_pool_map(&tk, k_cache, desc, 16)) != PKV_OK) return st;
+        if ((st = encode_pool_map(&tv, v_cache, desc, 16)) != PKV_OK) return st;
+        BalancedArgs a = {};
+        a.out = out;
+        a.q = q;
+        a.block_tables = block_tables;
+        a.context_lens = context_lens;
+        a.ws_o = static_cast<float*>(workspace);
+        a.ws_ml = a.ws_o + static_cast<int64_t>(grid) * 2 * group * desc->head_dim;
+        a.ws_meta = reinterpret_cast<int32_t*>(a.ws_ml + static_cast<int64_t>(grid) * 2 * group * 2);
+        a.err_flag = err_flag;
+        a.num_seqs = num_seqs;
+        a.num_heads = num_heads;
+        a.num_kv_heads = desc->num_kv_heads;
+        a.group = group;
+        a.max_blocks_per_seq = max_blocks_per_seq;
+        a.num_blocks = desc->num_blocks;
+        a.scale_log2 = scale * kLog2e;
+        return dispatch<RunBalanced>(desc, tk, tv, a, grid, smem, s);
+    }
+
     const int64_t max_len = static_cast<int64_t>(max_blocks_per_seq) * desc->block_size;
+    const bool split = partition_size < max_len;
     DecodeArgs a = {};
     a.out = out;
     a.q = q;
@@ -632,9 +1150,9 @@ extern "C" pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* o
     a.num_blocks = desc->num_blocks;
     a.scale_log2 = scale * kLog2e;
     if (split) {
-        const int64_t pmax = (max_len + P - 1) / P;
+        const int64_t pmax = (max_len + partition_size - 1) / partition_size;
         if (pmax > 65535) return fail(PKV_ERR_UNSUPPORTED, "too many partitions (> 65535)");
-        const size_t need = workspace_for(desc, num_seqs, num_heads, max_blocks_per_seq, P);
+        const size_t need = fixed_workspace(desc, num_seqs, num_heads, max_blocks_per_seq, partition_size);
         if (!workspace || workspace_bytes < need)
             return fail(PKV_ERR_WORKSPACE_TOO_SMALL, "paged_attention_decode: workspace too small");
         if (!aligned(workspace, 16))
@@ -643,19 +1161,15 @@ extern "C" pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* o
         a.ws_o = static_cast<float*>(workspace);
         a.ws_m = a.ws_o + rows * desc->head_dim;
         a.ws_l = a.ws_m + rows;
-        a.partition_tokens = P;
+        a.partition_tokens = partition_size;
         a.max_partitions = static_cast<int32_t>(pmax);
     } else {
         a.partition_tokens = static_cast<int32_t>(max_len);
         a.max_partitions = 1;
     }
-
-    CUtensorMap tk, tv;
-    if ((st = encode_pool_map(&tk, k_cache, desc)) != PKV_OK) return st;
-    if ((st = encode_pool_map(&tv, v_cache, desc)) != PKV_OK) return st;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (desc->dtype == PKV_BF16) return dispatch_shape<__nv_bfloat16>(desc, tk, tv, a, num_seqs, split, s);
-    return dispatch_shape<__half>(desc, tk, tv, a, num_seqs, split, s);
+    if ((st = encode_pool_map(&tk, k_cache, desc, desc->block_size)) != PKV_OK) return st;
+    if ((st = encode_pool_map(&tv, v_cache, desc, desc->block_size)) != PKV_OK) return st;
+    return dispatch<RunFixed>(desc, tk, tv, a, num_seqs, split, s);
 }
 
 // ------------------------------------------------ decode without allocation

@@ -334,3 +334,62 @@ def test_partial_shared_block_copy_on_write():
     wl.new_value = normal_tensor(rng, (n_new, wl.num_kv_heads, wl.head_dim), wl.dtype)
     pairs, *_ = _run_step(wl, None)
     assert len(pairs) == 3
+
+
+# ------------------------------------------------------------ balanced schedule
+
+@pytest.mark.parametrize("dtype,D,bs,group", [(torch.bfloat16, 128, 16, 4), (torch.float16, 64, 32, 8),
+                                              (torch.bfloat16, 128, 32, 8), (torch.bfloat16, 128, 16, 16),
+                                              (torch.float16, 64, 16, 1)])
+def test_balanced_many_short_and_empty_sequences(dtype, D, bs, group):
+    """Hundreds of (sequence, kv head) segments per CTA, some sequences empty."""
+    rng = np.random.default_rng(7)
+    lens = rng.integers(0, 60, size=700)
+    lens[::37] = 0
+    wl = custom_workload(num_seqs=700, num_heads=2 * group, num_kv_heads=2, head_dim=D, block_size=bs,
+                         context_lens=lens, dtype=dtype, seed=3)
+    dev = Dev(wl)
+    out = dev.decode(0)
+    assert dev.err.item() == 0
+    compare(out, oracle_decode(wl), what="balanced short")
+    assert torch.all(out[torch.from_numpy(lens == 0)] == 0)
+
+
+def test_balanced_one_long_sequence_is_chained_across_ctas():
+    wl = custom_workload(num_seqs=1, num_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+                         context_lens=[32768], seed=4)
+    dev = Dev(wl)
+    out = dev.decode(0)
+    assert dev.err.item() == 0
+    compare(out, oracle_decode(wl), what="balanced long")
+
+
+@pytest.mark.parametrize("lens", [[5, 40], [1], [0, 0, 17], [16, 0]])
+def test_balanced_fewer_units_than_ctas(lens):
+    wl = custom_workload(num_seqs=len(lens), num_heads=8, num_kv_heads=2, head_dim=128, block_size=16,
+                         context_lens=lens, seed=5, max_blocks_per_seq=8)
+    dev = Dev(wl)
+    out = dev.decode(0)
+    assert dev.err.item() == 0
+    compare(out, oracle_decode(wl), what=f"balanced {lens}")
+
+
+def test_balanced_large_batch():
+    """More sequences than threads in the prologue's scan (several per thread)."""
+    rng = np.random.default_rng(8)
+    lens = rng.integers(1, 50, size=3000)
+    wl = custom_workload(num_seqs=3000, num_heads=8, num_kv_heads=2, head_dim=128, block_size=16,
+                         context_lens=lens, seed=6)
+    dev = Dev(wl)
+    out = dev.decode(0)
+    assert dev.err.item() == 0
+    compare(out, oracle_decode(wl), what="balanced large batch")
+
+
+def test_balanced_full_size_long_context():
+    wl = make_workload(4, seed=0)
+    dev = Dev(wl)
+    out = dev.decode(0)
+    assert dev.err.item() == 0
+    seqs = _sample(wl, 3)
+    compare(out, oracle_decode(wl, seqs=seqs), seqs=seqs, what="config 4 balanced")
