@@ -293,6 +293,7 @@ __global__ void __launch_bounds__(D) reduce_kernel(const DecodeArgs a, int32_t m
 constexpr int kSegSlots = 4;          // segment descriptors in flight
 constexpr int kMergeSlots = 2;        // segments handed to the merge warp, in flight
 constexpr int kBalancedThreads = (kConsumerWarps + 2) * 32;  // + producer + merge warp
+constexpr int kMinUnits = 8;          // fewest units a CTA of the balanced grid takes
 constexpr int kMetaValid = 1;         // partial-slot meta flags
 constexpr int kMetaBegins = 2;        // the segment starts at the (b, hk)'s first block
 constexpr int kMetaEnds = 4;          // the segment ends at the (b, hk)'s last block
@@ -451,9 +452,12 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
     const long long excl = before + incl - mine;          // units (per kv head) before b_lo
     const long long units = total * Hkv;
-    // Spread the units over min(G, U) CTAs, so that every range is non-empty and
-    // the CTAs that share one (b, hk) are consecutive.
-    const long long used = units < grid ? units : grid;
+    // Spread the units over min(G, ceil(U / kMinUnits)) CTAs: every range is
+    // non-empty (at least kMinUnits units unless U is smaller), and the CTAs that
+    // share one (b, hk) are consecutive.  Small batches thus use fewer CTAs
+    // instead of splitting every sequence into one-unit pieces.
+    const long long want = (units + kMinUnits - 1) / kMinUnits;
+    const long long used = want < grid ? want : grid;
     const long long u0 = c < used ? static_cast<long long>(c) * units / used : 0;
     const long long u1 = c < used ? static_cast<long long>(c + 1) * units / used : 0;
     if (u0 < u1 && mine > 0 && excl * Hkv <= u0 && u0 < (excl + mine) * Hkv) {
@@ -778,59 +782,88 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 // Merge the partials of every (b, hk) that was split across CTAs.  CTA c owns
 // the chains that start in it (a partial marked "begins"); a chain continues in
-// slot 0 of CTAs c+1, c+2, ... until a partial marked "ends".  Sequences with
-// no tokens get zeros here.
+// slot 0 of CTAs c+1, c+2, ... up to the partial marked "ends".  Each chain is
+// merged in CTA order: M = max m_p, out = sum 2^(m_p - M) o_p / sum 2^(m_p - M) l_p.
+// Sequences with no tokens get zeros here.
+constexpr int kReduceThreads = 128;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(256) balanced_reduce_kernel(const BalancedArgs a) {
+__global__ void __launch_bounds__(kReduceThreads) balanced_reduce_kernel(const BalancedArgs a) {
     pdl_wait_primary();
+    __shared__ int s_chain_len;
     const int c = blockIdx.x;
     const int grid = gridDim.x;
     const int group = a.group;
+    const int tid = threadIdx.x;
     for (int slot = 0; slot < 2; ++slot) {
         const int32_t* meta = a.ws_meta + (static_cast<int64_t>(c) * 2 + slot) * 4;
         const int flags = meta[2];
-        if (!(flags & kMetaValid) || !(flags & kMetaBegins)) continue;
+        if (!(flags & kMetaValid) || !(flags & kMetaBegins)) continue;  // uniform over the CTA
         const int b = meta[0], hk = meta[1];
-        for (int idx = threadIdx.x; idx < group * D; idx += blockDim.x) {
-            const int r = idx / D;
-            const int d = idx - r * D;
-            // the chain's length: up to and including the partial marked "ends"
-            int last = c;
-            bool broken = false;
-            if (!(flags & kMetaEnds)) {
-                for (;;) {
-                    ++last;
-                    const int32_t* nm = a.ws_meta + static_cast<int64_t>(last) * 8;
-                    if (last >= grid || !(nm[2] & kMetaValid) || nm[0] != b || nm[1] != hk) {
-                        broken = true;
-                        --last;
-                        break;
+        if (tid < 32) {
+            // the chain's length: the first of CTAs c+1, c+2, ... whose slot 0 "ends"
+            int len = 0;
+            for (int base_c = c + 1; len == 0; base_c += 32) {
+                const int cc = base_c + tid;
+                int status = 0;  // 1: continues, 2: ends here, 3: broken
+                if (cc < grid) {
+                    const int32_t* nm = a.ws_meta + static_cast<int64_t>(cc) * 8;
+                    const int nf = nm[2];
+                    status = (!(nf & kMetaValid) || nm[0] != b || nm[1] != hk) ? 3 : ((nf & kMetaEnds) ? 2 : 1);
+                } else {
+                    status = 3;
+                }
+                const unsigned stop = __ballot_sync(0xffffffffu, status >= 2);
+                if (stop) {
+                    const int first = __ffs(stop) - 1;
+                    const int st_first = __shfl_sync(0xffffffffu, status, first);
+                    len = base_c + first - c + 1;
+                    if (st_first == 3) {  // a CTA of the chain is missing: keep what is there
+                        len -= 1;
+                        if (tid == 0) flag(a.err_flag, PKV_DEVERR_WAIT_TIMEOUT);
                     }
-                    if (nm[2] & kMetaEnds) break;
                 }
             }
-            if (broken && d == 0 && r == 0) flag(a.err_flag, PKV_DEVERR_WAIT_TIMEOUT);
+            if (tid == 0) s_chain_len = len;
+        }
+        __syncthreads();
+        const int n = s_chain_len;
+        // (row, 4 columns) per thread
+        for (int item = tid; item < group * (D / 4); item += kReduceThreads) {
+            const int r = item / (D / 4);
+            const int d0 = (item - r * (D / 4)) * 4;
             float M = -INFINITY;
-            for (int cc = c; cc <= last; ++cc) {
-                const int64_t p = static_cast<int64_t>(cc) * 2 + (cc == c ? slot : 0);
+            for (int k = 0; k < n; ++k) {
+                const int64_t p = static_cast<int64_t>(c + k) * 2 + (k == 0 ? slot : 0);
                 M = fmaxf(M, a.ws_ml[(p * group + r) * 2]);
             }
-            float acc = 0.f, den = 0.f;
-            for (int cc = c; cc <= last; ++cc) {
-                const int64_t p = static_cast<int64_t>(cc) * 2 + (cc == c ? slot : 0);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            float den = 0.f;
+            for (int k = 0; k < n; ++k) {
+                const int64_t p = static_cast<int64_t>(c + k) * 2 + (k == 0 ? slot : 0);
                 const float f = exp2_approx(a.ws_ml[(p * group + r) * 2] - M);
-                acc += f * a.ws_o[(p * group + r) * D + d];
+                const float4 o = *reinterpret_cast<const float4*>(a.ws_o + (p * group + r) * D + d0);
+                acc.x += f * o.x;
+                acc.y += f * o.y;
+                acc.z += f * o.z;
+                acc.w += f * o.w;
                 den += f * a.ws_ml[(p * group + r) * 2 + 1];
             }
+            const float inv = den > 0.f ? 1.f / den : 0.f;
+            float r0, r1;
+            uint2 packed;
+            packed.x = Pack<T>::two(acc.x * inv, acc.y * inv, r0, r1);
+            packed.y = Pack<T>::two(acc.z * inv, acc.w * inv, r0, r1);
             const int64_t bh = static_cast<int64_t>(b) * a.num_heads + static_cast<int64_t>(hk) * group + r;
-            static_cast<T*>(a.out)[bh * D + d] = Pack<T>::one(den > 0.f ? acc / den : 0.f);
+            *reinterpret_cast<uint2*>(static_cast<T*>(a.out) + bh * D + d0) = packed;
         }
+        __syncthreads();
     }
     // sequences with no tokens: zeros (context lengths <= 0 count as empty)
     for (int b = c; b < a.num_seqs; b += grid) {
         if (__ldg(a.context_lens + b) > 0) continue;
         T* o = static_cast<T*>(a.out) + static_cast<int64_t>(b) * a.num_heads * D;
-        for (int idx = threadIdx.x; idx < a.num_heads * D; idx += blockDim.x) o[idx] = Pack<T>::one(0.f);
+        for (int idx = tid; idx < a.num_heads * D; idx += kReduceThreads) o[idx] = Pack<T>::one(0.f);
     }
 }
 
@@ -986,7 +1019,7 @@ pkv_status launch_balanced(const CUtensorMap& tk, const CUtensorMap& tv, const B
     if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    cfg.blockDim = dim3(256);
+    cfg.blockDim = dim3(kReduceThreads);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
