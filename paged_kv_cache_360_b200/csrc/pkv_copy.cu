@@ -25,6 +25,8 @@ append_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
               const int64_t* __restrict__ slot_mapping, int64_t total_chunks,
               int32_t chunks_per_row, int32_t num_kv_heads, int32_t block_size,
               int64_t num_slots, int32_t* err_flag) {
+    // let a decode launched behind this kernel start its set-up now
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_chunks;
          i += stride) {

@@ -43,6 +43,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <utility>
 
 #include "pkv.h"
 #include "pkv_attend.cuh"
@@ -145,6 +146,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const int hk = blockIdx.x - b * a.num_kv_heads;
     const int part = blockIdx.y;
 
+    // Launched as a programmatic dependent of the previous kernel in the stream
+    // (e.g. the append): nothing global is touched before that kernel is done.
+    pdl_wait_primary();
     if (SPLIT) pdl_launch_dependents();
 
     const int max_len = a.max_blocks_per_seq * BS;
@@ -423,6 +427,9 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int Hkv = a.num_kv_heads;
     const int max_len = a.max_blocks_per_seq * BS;
 
+    // Launched as a programmatic dependent of the previous kernel in the stream
+    // (e.g. the append): nothing global is touched before that kernel is done.
+    pdl_wait_primary();
     pdl_launch_dependents();
     if (tid < 8) a.ws_meta[static_cast<int64_t>(c) * 8 + tid] = 0;  // both partial slots invalid
 
@@ -786,49 +793,81 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 // merged in CTA order: M = max m_p, out = sum 2^(m_p - M) o_p / sum 2^(m_p - M) l_p.
 // Sequences with no tokens get zeros here.
 constexpr int kReduceThreads = 128;
+constexpr int kChainWindow = 32;  // chains up to this many CTAs long are found in one round
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kReduceThreads) balanced_reduce_kernel(const BalancedArgs a) {
-    pdl_wait_primary();
-    __shared__ int s_chain_len;
+    __shared__ int s_meta[2 + kChainWindow][3];  // own slots 0 and 1, then slot 0 of c+1 ..
+    __shared__ int s_len[2];
     const int c = blockIdx.x;
     const int grid = gridDim.x;
     const int group = a.group;
     const int tid = threadIdx.x;
-    for (int slot = 0; slot < 2; ++slot) {
-        const int32_t* meta = a.ws_meta + (static_cast<int64_t>(c) * 2 + slot) * 4;
-        const int flags = meta[2];
-        if (!(flags & kMetaValid) || !(flags & kMetaBegins)) continue;  // uniform over the CTA
-        const int b = meta[0], hk = meta[1];
-        if (tid < 32) {
-            // the chain's length: the first of CTAs c+1, c+2, ... whose slot 0 "ends"
-            int len = 0;
-            for (int base_c = c + 1; len == 0; base_c += 32) {
-                const int cc = base_c + tid;
-                int status = 0;  // 1: continues, 2: ends here, 3: broken
-                if (cc < grid) {
-                    const int32_t* nm = a.ws_meta + static_cast<int64_t>(cc) * 8;
-                    const int nf = nm[2];
-                    status = (!(nf & kMetaValid) || nm[0] != b || nm[1] != hk) ? 3 : ((nf & kMetaEnds) ? 2 : 1);
-                } else {
-                    status = 3;
-                }
-                const unsigned stop = __ballot_sync(0xffffffffu, status >= 2);
-                if (stop) {
-                    const int first = __ffs(stop) - 1;
-                    const int st_first = __shfl_sync(0xffffffffu, status, first);
-                    len = base_c + first - c + 1;
-                    if (st_first == 3) {  // a CTA of the chain is missing: keep what is there
-                        len -= 1;
-                        if (tid == 0) flag(a.err_flag, PKV_DEVERR_WAIT_TIMEOUT);
-                    }
-                }
-            }
-            if (tid == 0) s_chain_len = len;
+
+    // The lengths are an input of the whole step (ready before the decode
+    // started), so they are read before waiting for the decode's results.
+    bool empty_seq[4] = {false, false, false, false};
+    {
+        int k = 0;
+        for (int b = c; b < a.num_seqs && k < 4; b += grid, ++k) empty_seq[k] = __ldg(a.context_lens + b) <= 0;
+    }
+
+    pdl_wait_primary();  // the decode's partials and descriptors are visible after this
+    if (tid < 2 + kChainWindow) {
+        const int cc = tid < 2 ? c : c + tid - 1;
+        const int slot = tid == 1 ? 1 : 0;
+        int m0 = 0, m1 = 0, m2 = 0;
+        if (cc < grid) {
+            const int32_t* m = a.ws_meta + (static_cast<int64_t>(cc) * 2 + slot) * 4;
+            m0 = m[0];
+            m1 = m[1];
+            m2 = m[2];
         }
-        __syncthreads();
-        const int n = s_chain_len;
-        // (row, 4 columns) per thread
+        s_meta[tid][0] = m0;
+        s_meta[tid][1] = m1;
+        s_meta[tid][2] = m2;
+    }
+    __syncthreads();
+    if (tid < 2) {
+        // chain starting in this CTA's slot `tid`: it continues in slot 0 of
+        // c+1, c+2, ... up to the partial marked "ends"
+        int len = 0;
+        const int f = s_meta[tid][2];
+        if ((f & kMetaValid) && (f & kMetaBegins)) {
+            const int b = s_meta[tid][0], hk = s_meta[tid][1];
+            len = 1;
+            for (int k = 1;; ++k) {
+                int nf, nb, nhk;
+                if (k <= kChainWindow) {
+                    nb = s_meta[k + 1][0];
+                    nhk = s_meta[k + 1][1];
+                    nf = s_meta[k + 1][2];
+                } else if (c + k < grid) {
+                    const int32_t* m = a.ws_meta + static_cast<int64_t>(c + k) * 8;
+                    nb = m[0];
+                    nhk = m[1];
+                    nf = m[2];
+                } else {
+                    nf = 0;
+                    nb = nhk = -1;
+                }
+                if (!(nf & kMetaValid) || nb != b || nhk != hk) {  // a CTA of the chain is missing
+                    flag(a.err_flag, PKV_DEVERR_WAIT_TIMEOUT);
+                    break;
+                }
+                ++len;
+                if (nf & kMetaEnds) break;
+            }
+        }
+        s_len[tid] = len;
+    }
+    __syncthreads();
+
+    for (int slot = 0; slot < 2; ++slot) {
+        const int n = s_len[slot];
+        if (n == 0) continue;
+        const int b = s_meta[slot][0], hk = s_meta[slot][1];
+        // (row, 4 columns) per thread: M = max m_p, out = sum 2^(m_p - M) o_p / sum 2^(m_p - M) l_p
         for (int item = tid; item < group * (D / 4); item += kReduceThreads) {
             const int r = item / (D / 4);
             const int d0 = (item - r * (D / 4)) * 4;
@@ -857,11 +896,13 @@ __global__ void __launch_bounds__(kReduceThreads) balanced_reduce_kernel(const B
             const int64_t bh = static_cast<int64_t>(b) * a.num_heads + static_cast<int64_t>(hk) * group + r;
             *reinterpret_cast<uint2*>(static_cast<T*>(a.out) + bh * D + d0) = packed;
         }
-        __syncthreads();
     }
+
     // sequences with no tokens: zeros (context lengths <= 0 count as empty)
-    for (int b = c; b < a.num_seqs; b += grid) {
-        if (__ldg(a.context_lens + b) > 0) continue;
+    int k = 0;
+    for (int b = c; b < a.num_seqs; b += grid, ++k) {
+        const bool empty = k < 4 ? empty_seq[k] : __ldg(a.context_lens + b) <= 0;
+        if (!empty) continue;
         T* o = static_cast<T*>(a.out) + static_cast<int64_t>(b) * a.num_heads * D;
         for (int idx = tid; idx < a.num_heads * D; idx += kReduceThreads) o[idx] = Pack<T>::one(0.f);
     }
@@ -946,6 +987,25 @@ cudaError_t opt_in_smem(const void* kernel) {
     return e;
 }
 
+// Launch `kernel` as a programmatic dependent of the previous work in `stream`:
+// it may start while that work finishes, and waits for it in
+// griddepcontrol.wait before touching global memory.
+template <typename... P, typename... A>
+cudaError_t launch_dependent(void (*kernel)(P...), dim3 grid, dim3 block, int smem,
+                             cudaStream_t stream, A&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
+
 template <typename T, int D, int BS, bool SPLIT>
 struct FixedTag {};
 template <typename T, int D, int BS>
@@ -962,9 +1022,9 @@ pkv_status launch_fixed(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
         auto k = decode_kernel<T, D, BS, true>;
         if ((e = opt_in_smem<FixedTag<T, D, BS, true>>(reinterpret_cast<const void*>(k))) != cudaSuccess)
             return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
-        k<<<grid, kThreads, Lay::kSmemBytes, stream>>>(tk, tv, a);
+        e = launch_dependent(k, grid, dim3(kThreads), Lay::kSmemBytes, stream, tk, tv, a);
         note_launches(1);
-        if ((e = cudaGetLastError()) != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+        if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
         // The merge launches as a programmatic dependent of the partition
         // kernel: its CTAs may start during the partition kernel's tail and wait
         // in griddepcontrol.wait for the results.
@@ -985,9 +1045,9 @@ pkv_status launch_fixed(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
         auto k = decode_kernel<T, D, BS, false>;
         if ((e = opt_in_smem<FixedTag<T, D, BS, false>>(reinterpret_cast<const void*>(k))) != cudaSuccess)
             return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
-        k<<<grid, kThreads, Lay::kSmemBytes, stream>>>(tk, tv, a);
+        e = launch_dependent(k, grid, dim3(kThreads), Lay::kSmemBytes, stream, tk, tv, a);
         note_launches(1);
-        if ((e = cudaGetLastError()) != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+        if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
     }
     return PKV_OK;
 }
@@ -995,7 +1055,18 @@ pkv_status launch_fixed(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
 // Resident CTAs of the balanced kernel on the current device: its grid size.
 template <typename T, int D, int BS>
 pkv_status balanced_grid(int group, int* grid_out, int* smem_out) {
+    // resident CTAs per (device, group), computed once
+    static std::atomic<int> cache[64][17];
     const BalancedLayout<D> lay(group);
+    int dev0 = 0;
+    if (cudaGetDevice(&dev0) == cudaSuccess && dev0 >= 0 && dev0 < 64 && group >= 1 && group <= 16) {
+        const int g = cache[dev0][group].load(std::memory_order_acquire);
+        if (g > 0) {
+            *grid_out = g;
+            *smem_out = lay.total;
+            return PKV_OK;
+        }
+    }
     auto k = balanced_kernel<T, D, BS>;
     cudaError_t e = opt_in_smem<BalancedTag<T, D, BS>>(reinterpret_cast<const void*>(k));
     if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
@@ -1007,15 +1078,17 @@ pkv_status balanced_grid(int group, int* grid_out, int* smem_out) {
     if (per_sm < 1) return fail(PKV_ERR_UNSUPPORTED, "balanced decode does not fit on an SM");
     *grid_out = sms * per_sm;
     *smem_out = lay.total;
+    if (dev >= 0 && dev < 64 && group >= 1 && group <= 16)
+        cache[dev][group].store(*grid_out, std::memory_order_release);
     return PKV_OK;
 }
 
 template <typename T, int D, int BS>
 pkv_status launch_balanced(const CUtensorMap& tk, const CUtensorMap& tv, const BalancedArgs& a,
                            int grid, int smem, cudaStream_t stream) {
-    balanced_kernel<T, D, BS><<<grid, kBalancedThreads, smem, stream>>>(tk, tv, a);
+    cudaError_t e = launch_dependent(balanced_kernel<T, D, BS>, dim3(grid), dim3(kBalancedThreads), smem,
+                                     stream, tk, tv, a);
     note_launches(1);
-    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
