@@ -109,6 +109,24 @@ pkv_status copy_blocks(const pkv_cache_desc* desc, void* k_cache, void* v_cache,
                        void* stream);
 
 /*
+ * Swap blocks between the pools and host memory, for preemption by swapping
+ * ([ops page] How it works: a preempted sequence's blocks are swapped to host
+ * memory and restored later).
+ *   block_list  device int32 [n]: physical block ids.
+ *   host_k, host_v  page-locked host memory (cudaHostAlloc / cudaMallocHost,
+ *               torch pin_memory), [n][num_kv_heads][block_size][head_dim]
+ *               elements each; the kernel reads or writes it directly over the
+ *               host link.  Pageable memory is refused (PKV_ERR_INVALID_ARG).
+ *   to_host     1: host[i] = pool[block_list[i]] (swap out);
+ *               0: pool[block_list[i]] = host[i] (swap in).
+ *   err_flag    device int32 or NULL; PKV_DEVERR_BAD_PAIR for an id outside the pool.
+ * n == 0 enqueues nothing.  Bit-exact.
+ */
+pkv_status swap_blocks(const pkv_cache_desc* desc, void* k_cache, void* v_cache, void* host_k,
+                       void* host_v, const int32_t* block_list, int32_t n, int32_t to_host,
+                       int32_t* err_flag, void* stream);
+
+/*
  * Workspace bytes paged_attention_decode needs for these shapes and
  * partition_size.
  *   partition_size 0 (balanced): 2 * G * (group * (head_dim + 2) * 4 + 16) bytes,
@@ -227,7 +245,8 @@ typedef struct pkv_stats {
     int64_t live_slots;      /* distinct slots holding a token of a live sequence    */
     int64_t live_tokens;     /* sum of live sequence lengths (shared tokens counted per sequence) */
     int64_t shared_blocks;   /* blocks with reference count > 1                      */
-    int64_t num_seqs;        /* live sequences                                       */
+    int64_t num_seqs;        /* resident (not swapped-out) sequences                 */
+    int64_t swapped_seqs;    /* swapped-out sequences                                */
 } pkv_stats;
 
 /* free_order: host int32 [num_blocks], a permutation of 0..num_blocks-1, or NULL. */
@@ -262,6 +281,27 @@ pkv_status pkv_seq_cow(pkv_pool* pool, int32_t seq, int32_t logical_block, int32
 
 /* Release the sequence: every block's refcount - 1; blocks reaching 0 return to the pool. */
 pkv_status pkv_seq_free(pkv_pool* pool, int32_t seq);
+
+/*
+ * Preemption by swapping ([ops page] How it works: when the free pool empties
+ * the scheduler preempts a sequence and swaps its blocks to host memory, then
+ * restores them later).
+ * pkv_seq_swap_out: write the sequence's blocks, logical order, to blocks_out
+ * (host int32, capacity cap >= its block count; *n = the count), then release
+ * them exactly as pkv_seq_free does.  The sequence keeps its length and id and
+ * holds no blocks; reserve, fork, cow and pkv_pool_block_tables refuse it until
+ * it is swapped in.  Copy the listed blocks out (swap_blocks, device to host)
+ * before anything reuses them.
+ * pkv_seq_swap_in: take ceil(len / block_size) fresh blocks, all or nothing
+ * (PKV_ERR_NO_FREE_BLOCK and no change if the pool is short), make them the
+ * sequence's table and write them, logical order, to blocks_out; then copy the
+ * saved contents back into them (swap_blocks, host to device).  Sharing is not
+ * restored: every block comes back with reference count 1.
+ */
+pkv_status pkv_seq_swap_out(pkv_pool* pool, int32_t seq, int32_t* blocks_out, int32_t cap,
+                            int32_t* n);
+pkv_status pkv_seq_swap_in(pkv_pool* pool, int32_t seq, int32_t* blocks_out, int32_t cap,
+                           int32_t* n);
 
 pkv_status pkv_seq_len(const pkv_pool* pool, int32_t seq, int64_t* len);
 

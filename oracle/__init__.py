@@ -68,6 +68,8 @@ def _load():
             lib.oracle_append.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i32]
             lib.oracle_copy_blocks.restype = ctypes.c_int
             lib.oracle_copy_blocks.argtypes = [p, p, p, i32, i32, i32, i32, i32]
+            lib.oracle_swap_blocks.restype = ctypes.c_int
+            lib.oracle_swap_blocks.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i32, i32]
             _lib = lib
     return _lib
 
@@ -171,6 +173,21 @@ def copy_blocks(k_words: np.ndarray, v_words: np.ndarray, block_mapping) -> None
                                     D, bs, NB)
     if rc != 0:
         raise ValueError(f"oracle_copy_blocks failed ({rc})")
+
+
+def swap_blocks(k_words: np.ndarray, v_words: np.ndarray, host_k: np.ndarray, host_v: np.ndarray,
+                block_list, to_host: bool) -> None:
+    """Swap out (to_host) or in whole blocks between uint16 pools [NB, Hkv, bs, D]
+    and uint16 host buffers [n, Hkv, bs, D]; all arrays modified in place."""
+    NB, Hkv, bs, D = k_words.shape
+    blocks = np.ascontiguousarray(block_list, dtype=np.int32)
+    for a in (k_words, v_words, host_k, host_v):
+        assert a.dtype == np.uint16 and a.flags.c_contiguous
+    assert host_k.shape[0] >= len(blocks) and host_v.shape[0] >= len(blocks)
+    rc = _load().oracle_swap_blocks(_ptr(k_words), _ptr(v_words), _ptr(host_k), _ptr(host_v),
+                                    _ptr(blocks), len(blocks), 1 if to_host else 0, Hkv, D, bs, NB)
+    if rc != 0:
+        raise ValueError(f"oracle_swap_blocks failed ({rc})")
 
 
 words = _words

@@ -32,6 +32,18 @@ can be compared exactly; any order is correct by the pages):
 * ``cow(seq, i)`` gives the sequence a private copy of logical block i when the
   block is shared, and does nothing otherwise;
 * a slot id is ``physical_block * block_size + offset``.
+
+Preemption by swapping ("PagedAttention" ops page, How it works: when the free
+pool empties the scheduler preempts a sequence and swaps its blocks to host
+memory, then restores them later):
+
+* ``swap_out(seq)`` returns the sequence's blocks in logical order (the caller
+  copies them to host memory) and releases them exactly as ``free_seq`` would;
+  the sequence keeps its length and holds no blocks while swapped;
+* ``swap_in(seq)`` takes ``ceil(len / block_size)`` fresh blocks from the pool,
+  all or nothing, and returns them in logical order (the caller copies the saved
+  contents back into them); sharing is not restored: every block comes back
+  private.
 """
 
 from __future__ import annotations
@@ -60,12 +72,18 @@ class BlockPoolModel:
     def new_seq(self) -> int:
         sid = self.next_id
         self.next_id += 1
-        self.seqs[sid] = {"blocks": [], "len": 0}
+        self.seqs[sid] = {"blocks": [], "len": 0, "swapped": False}
         return sid
+
+    def _resident(self, sid):
+        seq = self.seqs[sid]
+        if seq["swapped"]:
+            raise ValueError(f"sequence {sid} is swapped out")
+        return seq
 
     def fork(self, parent: int) -> int:
         """A new sequence that shares every block of ``parent`` (refcount + 1 each)."""
-        src = self.seqs[parent]
+        src = self._resident(parent)
         sid = self.new_seq()
         self.seqs[sid]["blocks"] = list(src["blocks"])
         self.seqs[sid]["len"] = src["len"]
@@ -80,7 +98,7 @@ class BlockPoolModel:
 
     def reserve(self, sid: int, n_tokens: int):
         """Make room for ``n_tokens`` more tokens; return (slots, cow_pairs)."""
-        seq = self.seqs[sid]
+        seq = self._resident(sid)
         bs = self.block_size
         length = seq["len"]
         # Count what the request needs before touching anything.
@@ -117,7 +135,7 @@ class BlockPoolModel:
 
     def cow(self, sid: int, logical_block: int):
         """Give ``sid`` a private copy of one shared block; return the pair or None."""
-        seq = self.seqs[sid]
+        seq = self._resident(sid)
         cur = seq["blocks"][logical_block]
         if self.refcount[cur] <= 1:
             return None
@@ -128,12 +146,36 @@ class BlockPoolModel:
         seq["blocks"][logical_block] = fresh
         return (cur, fresh)
 
-    def free_seq(self, sid: int) -> None:
-        seq = self.seqs.pop(sid)
-        for b in seq["blocks"]:
+    def _release(self, blocks) -> None:
+        for b in blocks:
             self.refcount[b] -= 1
             if self.refcount[b] == 0:
                 self.free.append(b)
+
+    def free_seq(self, sid: int) -> None:
+        seq = self.seqs.pop(sid)
+        self._release(seq["blocks"])
+
+    def swap_out(self, sid: int):
+        """Release the sequence's blocks to the pool; return them (logical order)."""
+        seq = self._resident(sid)
+        blocks = list(seq["blocks"])
+        self._release(blocks)
+        seq["blocks"] = []
+        seq["swapped"] = True
+        return blocks
+
+    def swap_in(self, sid: int):
+        """Give a swapped sequence fresh blocks for its whole length; return them."""
+        seq = self.seqs[sid]
+        if not seq["swapped"]:
+            raise ValueError(f"sequence {sid} is not swapped out")
+        need = -(-seq["len"] // self.block_size)
+        if need > len(self.free):
+            raise PoolExhausted(f"need {need} blocks, {len(self.free)} free")
+        seq["blocks"] = [self._pop() for _ in range(need)]
+        seq["swapped"] = False
+        return list(seq["blocks"])
 
     # -- views ---------------------------------------------------------------
     def table(self, sid: int):
@@ -149,7 +191,8 @@ class BlockPoolModel:
     def stats(self) -> dict:
         bs = self.block_size
         live = set()
-        for seq in self.seqs.values():
+        resident = [seq for seq in self.seqs.values() if not seq["swapped"]]
+        for seq in resident:
             for t in range(seq["len"]):
                 live.add((seq["blocks"][t // bs], t % bs))
         allocated = self.num_blocks - len(self.free)
@@ -157,9 +200,10 @@ class BlockPoolModel:
             "free_blocks": len(self.free),
             "allocated_slots": allocated * bs,
             "live_slots": len(live),
-            "live_tokens": sum(s["len"] for s in self.seqs.values()),
+            "live_tokens": sum(s["len"] for s in resident),
             "shared_blocks": sum(1 for r in self.refcount if r > 1),
-            "num_seqs": len(self.seqs),
+            "num_seqs": len(resident),
+            "swapped_seqs": len(self.seqs) - len(resident),
         }
 
 

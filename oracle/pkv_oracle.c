@@ -309,3 +309,31 @@ int oracle_copy_blocks(uint16_t* k_cache, uint16_t* v_cache, const int32_t* bloc
     }
     return 0;
 }
+
+/*
+ * Swap out: host[i] = pool[block_list[i]] for K and V, whole blocks ([ops page]
+ * How it works: a preempted sequence's blocks are swapped to host memory).
+ * Swap in: pool[block_list[i]] = host[i] (restored later).  host_k, host_v:
+ * [n][Hkv][bs][D] words.  Returns 0, or -1 if an id is outside the pool.
+ */
+int oracle_swap_blocks(uint16_t* k_cache, uint16_t* v_cache, uint16_t* host_k, uint16_t* host_v,
+                       const int32_t* block_list, int32_t n, int32_t to_host, int32_t Hkv,
+                       int32_t D, int32_t block_size, int32_t num_blocks) {
+    int64_t block_words = (int64_t)Hkv * block_size * D;
+    for (int32_t i = 0; i < n; ++i) {
+        int32_t blk = block_list[i];
+        if (blk < 0 || blk >= num_blocks) return -1;
+        uint16_t* pk = k_cache + blk * block_words;
+        uint16_t* pv = v_cache + blk * block_words;
+        uint16_t* hk = host_k + i * block_words;
+        uint16_t* hv = host_v + i * block_words;
+        if (to_host) {
+            memcpy(hk, pk, sizeof(uint16_t) * (size_t)block_words);
+            memcpy(hv, pv, sizeof(uint16_t) * (size_t)block_words);
+        } else {
+            memcpy(pk, hk, sizeof(uint16_t) * (size_t)block_words);
+            memcpy(pv, hv, sizeof(uint16_t) * (size_t)block_words);
+        }
+    }
+    return 0;
+}

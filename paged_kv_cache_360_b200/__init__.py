@@ -19,7 +19,8 @@ from . import _lib
 from ._lib import PkvError, PoolExhausted  # noqa: F401
 
 __all__ = [
-    "paged_kv_append", "copy_blocks", "paged_attention_decode", "paged_attention_workspace_bytes",
+    "paged_kv_append", "copy_blocks", "swap_blocks", "paged_attention_decode",
+    "paged_attention_workspace_bytes",
     "paged_attention_decode_static_scratch", "Pool",
     "PkvError", "PoolExhausted", "launch_count", "cache_desc",
 ]
@@ -91,6 +92,26 @@ def copy_blocks(k_cache, v_cache, block_mapping, err_flag=None, stream=None):
         _dev(err_flag, "err_flag", torch.int32), _stream(stream)))
 
 
+def swap_blocks(k_cache, v_cache, host_k, host_v, block_list, to_host: bool, err_flag=None,
+                stream=None):
+    """Copy whole blocks between the pools and page-locked host buffers
+    [n, num_kv_heads, block_size, head_dim]: host[i] = pool[block_list[i]] when
+    to_host, else pool[block_list[i]] = host[i].  block_list: int32 CUDA tensor [n]."""
+    torch = _torch()
+    desc = cache_desc(k_cache)
+    n = int(block_list.shape[0])
+    for name, t in (("host_k", host_k), ("host_v", host_v)):
+        if t.is_cuda or not t.is_pinned() or not t.is_contiguous() or t.dtype != k_cache.dtype:
+            raise PkvError(1, f"{name} must be contiguous page-locked host memory of the cache dtype")
+        if t.dim() != 4 or t.shape[0] < n or tuple(t.shape[1:]) != tuple(k_cache.shape[1:]):
+            raise PkvError(1, f"{name} must be [>= n, num_kv_heads, block_size, head_dim]")
+    _lib.check(_lib.load().swap_blocks(
+        ctypes.byref(desc), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        ctypes.c_void_p(host_k.data_ptr()), ctypes.c_void_p(host_v.data_ptr()),
+        _dev(block_list, "block_list", torch.int32), n, 1 if to_host else 0,
+        _dev(err_flag, "err_flag", torch.int32), _stream(stream)))
+
+
 def paged_attention_workspace_bytes(k_cache, num_seqs: int, num_heads: int,
                                     max_blocks_per_seq: int, partition_size: int = 0) -> int:
     desc = cache_desc(k_cache)
@@ -113,9 +134,10 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
     if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape[0] != B:
         raise PkvError(1, "block_tables must be [B, MB] and context_lens [B]")
     MB = int(block_tables.shape[1])
-    need = paged_attention_workspace_bytes(k_cache, B, H, MB, partition_size)
-    if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is None:
+        need = paged_attention_workspace_bytes(k_cache, B, H, MB, partition_size)
+        if need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _lib.check(_lib.load().paged_attention_decode(
         ctypes.byref(desc), _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"),
@@ -206,6 +228,24 @@ class Pool:
 
     def free_seq(self, seq: int) -> None:
         _lib.check(self._lib.pkv_seq_free(self._h, seq))
+
+    def swap_out(self, seq: int):
+        """Release the sequence's blocks (preemption); returns them, logical order."""
+        n = ctypes.c_int32()
+        cap = max(1, len(self.table(seq)))
+        out = np.empty(cap, dtype=np.int32)
+        _lib.check(self._lib.pkv_seq_swap_out(self._h, seq, out.ctypes.data_as(ctypes.c_void_p), cap,
+                                              ctypes.byref(n)))
+        return [int(x) for x in out[:n.value]]
+
+    def swap_in(self, seq: int):
+        """Fresh blocks for a swapped-out sequence (all or nothing); returns them."""
+        n = ctypes.c_int32()
+        cap = max(1, -(-self.length(seq) // self.block_size))
+        out = np.empty(cap, dtype=np.int32)
+        _lib.check(self._lib.pkv_seq_swap_in(self._h, seq, out.ctypes.data_as(ctypes.c_void_p), cap,
+                                             ctypes.byref(n)))
+        return [int(x) for x in out[:n.value]]
 
     def length(self, seq: int) -> int:
         n = ctypes.c_int64()

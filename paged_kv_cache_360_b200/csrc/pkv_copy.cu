@@ -71,7 +71,43 @@ copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
         to[i] = from[i];
 }
 
+// grid = (list entry i, pool [0 = K, 1 = V], slice): block list[i] of the pool
+// and entry i of the page-locked host buffer, copied in the `to_host` direction.
+__global__ void __launch_bounds__(kCopyThreads)
+swap_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache, uint4* host_k,
+                   uint4* host_v, const int32_t* __restrict__ block_list, int64_t block_chunks,
+                   int32_t num_blocks, int32_t to_host, int32_t* err_flag) {
+    const int32_t blk = __ldg(block_list + blockIdx.x);
+    if (blk < 0 || blk >= num_blocks) {
+        if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && err_flag)
+            atomicOr(err_flag, PKV_DEVERR_BAD_PAIR);
+        return;
+    }
+    uint4* dev = (blockIdx.y == 0 ? k_cache : v_cache) + static_cast<int64_t>(blk) * block_chunks;
+    uint4* host = (blockIdx.y == 0 ? host_k : host_v) + static_cast<int64_t>(blockIdx.x) * block_chunks;
+    const int64_t stride = static_cast<int64_t>(gridDim.z) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.z) * blockDim.x + threadIdx.x; i < block_chunks;
+         i += stride) {
+        if (to_host)
+            host[i] = dev[i];
+        else
+            dev[i] = host[i];
+    }
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The device address of page-locked host memory, or NULL for anything else
+// (pageable host memory must never reach a kernel).
+void* pinned_device_address(void* host) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, host) != cudaSuccess) {
+        cudaGetLastError();  // clear the error of an unknown pointer
+        return nullptr;
+    }
+    if (attr.type != cudaMemoryTypeHost) return nullptr;
+    return attr.devicePointer;
+}
 
 pkv_status check_desc(const pkv_cache_desc* d, const char* who) {
     if (!d) return fail(PKV_ERR_INVALID_ARG, who);
@@ -137,6 +173,35 @@ extern "C" pkv_status copy_blocks(const pkv_cache_desc* desc, void* k_cache, voi
     copy_blocks_kernel<<<grid, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), block_mapping, block_chunks,
         desc->num_blocks, err_flag);
+    note_launches(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+    return PKV_OK;
+}
+
+extern "C" pkv_status swap_blocks(const pkv_cache_desc* desc, void* k_cache, void* v_cache,
+                                  void* host_k, void* host_v, const int32_t* block_list, int32_t n,
+                                  int32_t to_host, int32_t* err_flag, void* stream) {
+    pkv_status st = check_desc(desc, "swap_blocks: desc is NULL");
+    if (st != PKV_OK) return st;
+    if (n < 0) return fail(PKV_ERR_INVALID_ARG, "swap_blocks: n < 0");
+    if (n == 0) return PKV_OK;
+    if (!k_cache || !v_cache || !host_k || !host_v || !block_list)
+        return fail(PKV_ERR_INVALID_ARG, "swap_blocks: NULL pointer");
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(host_k) || !aligned16(host_v))
+        return fail(PKV_ERR_INVALID_ARG, "swap_blocks: pools and host buffers must be 16-byte aligned");
+    void* dk = pinned_device_address(host_k);
+    void* dv = pinned_device_address(host_v);
+    if (!dk || !dv)
+        return fail(PKV_ERR_INVALID_ARG, "swap_blocks: host buffers must be page-locked host memory");
+    const int64_t block_chunks =
+        static_cast<int64_t>(desc->num_kv_heads) * desc->block_size * desc->head_dim * 2 / 16;
+    int64_t slices = (block_chunks + kCopyThreads * 4 - 1) / (kCopyThreads * 4);
+    if (slices > 65535) slices = 65535;
+    dim3 grid(static_cast<unsigned>(n), 2, static_cast<unsigned>(slices));
+    swap_blocks_kernel<<<grid, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<uint4*>(dk),
+        static_cast<uint4*>(dv), block_list, block_chunks, desc->num_blocks, to_host ? 1 : 0, err_flag);
     note_launches(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));

@@ -24,6 +24,7 @@ struct pkv_pool {
     std::vector<int32_t> refcount;
     struct Seq {
         bool live = false;
+        bool swapped = false;  // preempted: blocks given back, length kept
         int64_t len = 0;
         std::vector<int32_t> blocks;
     };
@@ -42,6 +43,15 @@ struct pkv_pool {
         free_stack.pop_back();
         refcount[b] = 1;
         return b;
+    }
+    Seq* resident(int32_t id) {
+        Seq* s = find(id);
+        return (s && !s->swapped) ? s : nullptr;
+    }
+    // refcount - 1 per block, logical order; blocks reaching 0 go on the free stack
+    void release(const std::vector<int32_t>& blocks) {
+        for (int32_t b : blocks)
+            if (--refcount[b] == 0) free_stack.push_back(b);
     }
 };
 
@@ -90,7 +100,8 @@ extern "C" pkv_status pkv_seq_new(pkv_pool* pool, int32_t* seq_id) {
 
 extern "C" pkv_status pkv_seq_fork(pkv_pool* pool, int32_t parent, int32_t* child) {
     if (!pool || !child) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_fork: NULL argument");
-    if (!pool->find(parent)) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_fork: unknown parent");
+    if (!pool->resident(parent))
+        return fail(PKV_ERR_INVALID_ARG, "pkv_seq_fork: unknown or swapped-out parent");
     pkv_pool::Seq copy = *pool->find(parent);
     for (int32_t b : copy.blocks) pool->refcount[b] += 1;
     pool->seqs.push_back(std::move(copy));
@@ -103,8 +114,8 @@ extern "C" pkv_status pkv_seq_reserve(pkv_pool* pool, int32_t seq, int32_t n_tok
                                       int32_t* n_cow_out) {
     if (!pool || n_tokens < 0 || (n_tokens > 0 && !slots_out))
         return fail(PKV_ERR_INVALID_ARG, "pkv_seq_reserve: bad argument");
-    pkv_pool::Seq* s = pool->find(seq);
-    if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_reserve: unknown sequence");
+    pkv_pool::Seq* s = pool->resident(seq);
+    if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_reserve: unknown or swapped-out sequence");
     const int64_t bs = pool->block_size;
     if (n_cow_out) *n_cow_out = 0;
     // Blocks needed: one per block boundary crossed, plus a copy if the first
@@ -144,8 +155,8 @@ extern "C" pkv_status pkv_seq_reserve(pkv_pool* pool, int32_t seq, int32_t n_tok
 extern "C" pkv_status pkv_seq_cow(pkv_pool* pool, int32_t seq, int32_t logical_block,
                                   int32_t* pair_out, int32_t* n_out) {
     if (!pool || !pair_out || !n_out) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_cow: NULL argument");
-    pkv_pool::Seq* s = pool->find(seq);
-    if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_cow: unknown sequence");
+    pkv_pool::Seq* s = pool->resident(seq);
+    if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_cow: unknown or swapped-out sequence");
     if (logical_block < 0 || logical_block >= static_cast<int32_t>(s->blocks.size()))
         return fail(PKV_ERR_INVALID_ARG, "pkv_seq_cow: logical block out of range");
     *n_out = 0;
@@ -166,13 +177,45 @@ extern "C" pkv_status pkv_seq_free(pkv_pool* pool, int32_t seq) {
     if (!pool) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_free: NULL pool");
     pkv_pool::Seq* s = pool->find(seq);
     if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_free: unknown sequence");
-    for (int32_t b : s->blocks) {
-        if (--pool->refcount[b] == 0) pool->free_stack.push_back(b);
-    }
+    pool->release(s->blocks);
     s->blocks.clear();
     s->blocks.shrink_to_fit();
     s->len = 0;
     s->live = false;
+    s->swapped = false;
+    return PKV_OK;
+}
+
+extern "C" pkv_status pkv_seq_swap_out(pkv_pool* pool, int32_t seq, int32_t* blocks_out, int32_t cap,
+                                       int32_t* n) {
+    if (!pool || !n) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_swap_out: NULL argument");
+    pkv_pool::Seq* s = pool->resident(seq);
+    if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_swap_out: unknown or swapped-out sequence");
+    const int32_t nb = static_cast<int32_t>(s->blocks.size());
+    if (cap < nb || (nb > 0 && !blocks_out))
+        return fail(PKV_ERR_INVALID_ARG, "pkv_seq_swap_out: blocks_out holds fewer than the sequence's blocks");
+    for (int32_t i = 0; i < nb; ++i) blocks_out[i] = s->blocks[i];
+    *n = nb;
+    pool->release(s->blocks);
+    s->blocks.clear();
+    s->swapped = true;
+    return PKV_OK;
+}
+
+extern "C" pkv_status pkv_seq_swap_in(pkv_pool* pool, int32_t seq, int32_t* blocks_out, int32_t cap,
+                                      int32_t* n) {
+    if (!pool || !n) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_swap_in: NULL argument");
+    pkv_pool::Seq* s = pool->find(seq);
+    if (!s || !s->swapped) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_swap_in: sequence is not swapped out");
+    const int64_t need = (s->len + pool->block_size - 1) / pool->block_size;
+    if (cap < need || (need > 0 && !blocks_out))
+        return fail(PKV_ERR_INVALID_ARG, "pkv_seq_swap_in: blocks_out holds fewer than the blocks needed");
+    if (need > static_cast<int64_t>(pool->free_stack.size()))
+        return fail(PKV_ERR_NO_FREE_BLOCK, "pkv_seq_swap_in: free pool exhausted");
+    for (int64_t i = 0; i < need; ++i) s->blocks.push_back(pool->pop());
+    for (int64_t i = 0; i < need; ++i) blocks_out[i] = s->blocks[i];
+    *n = static_cast<int32_t>(need);
+    s->swapped = false;
     return PKV_OK;
 }
 
@@ -204,7 +247,8 @@ extern "C" pkv_status pkv_pool_block_tables(const pkv_pool* pool, const int32_t*
         return fail(PKV_ERR_INVALID_ARG, "pkv_pool_block_tables: bad argument");
     for (int32_t i = 0; i < n_seqs; ++i) {
         const pkv_pool::Seq* s = pool->find(seqs[i]);
-        if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_pool_block_tables: unknown sequence");
+        if (!s || s->swapped)
+            return fail(PKV_ERR_INVALID_ARG, "pkv_pool_block_tables: unknown or swapped-out sequence");
         if (static_cast<int64_t>(s->blocks.size()) > max_blocks_per_seq)
             return fail(PKV_ERR_INVALID_ARG,
                         "pkv_pool_block_tables: a sequence has more blocks than max_blocks_per_seq");
@@ -244,9 +288,14 @@ extern "C" pkv_status pkv_pool_stats(const pkv_pool* pool, pkv_stats* st) {
     st->allocated_slots = (pool->num_blocks - st->free_blocks) * bs;
     st->live_tokens = 0;
     st->num_seqs = 0;
+    st->swapped_seqs = 0;
     std::unordered_set<int64_t> live;
     for (const auto& s : pool->seqs) {
         if (!s.live) continue;
+        if (s.swapped) {
+            st->swapped_seqs += 1;
+            continue;
+        }
         st->num_seqs += 1;
         st->live_tokens += s.len;
         for (int64_t t = 0; t < s.len; ++t) live.insert(static_cast<int64_t>(s.blocks[t / bs]) * bs + t % bs);

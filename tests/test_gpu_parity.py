@@ -9,6 +9,7 @@ five full-size workloads with the partition size the bench uses.  Block
 permutation and copy-on-write must leave the output bit-identical.
 """
 
+import ctypes
 import math
 
 import numpy as np
@@ -393,3 +394,88 @@ def test_balanced_full_size_long_context():
     assert dev.err.item() == 0
     seqs = _sample(wl, 3)
     compare(out, oracle_decode(wl, seqs=seqs), seqs=seqs, what="config 4 balanced")
+
+
+# ------------------------------------------------------------ swap (preemption)
+
+@pytest.mark.parametrize("dtype,D,bs", [(torch.bfloat16, 128, 16), (torch.float16, 64, 32)])
+def test_swap_out_and_in_through_the_block_manager(dtype, D, bs):
+    """Preempt a sequence (its blocks go to pinned host memory and back to the
+    pool), let another sequence reuse the blocks, restore it into fresh blocks:
+    the host copy, the pool after restore and the decode output all match the
+    oracle, and the output is bit-identical to the output before preemption."""
+    rng = np.random.default_rng(11)
+    Hkv, H, NB = 4, 16, 64
+    k, v, _ = _pool(12, NB, Hkv, bs, D, dtype)
+    pool = pkv.Pool(NB, bs, rng.permutation(NB))
+    model = oracle.BlockPoolModel(NB, bs, pool.free_list())
+    seqs = []
+    for L in (300, 77, 150):
+        a, b = pool.new_seq(), model.new_seq()
+        pool.reserve(a, L)
+        model.reserve(b, L)
+        seqs.append(a)
+    kd, vd = k.cuda(), v.cuda()
+    q = normal_tensor(rng, (3, H, D), dtype)
+    scale = float(np.float32(1.0 / np.sqrt(D)))
+
+    def decode():
+        mb = max(len(pool.table(s)) for s in seqs)
+        tables, lens = pool.block_tables(seqs, mb)
+        out = torch.empty((3, H, D), dtype=dtype, device="cuda")
+        pkv.paged_attention_decode(out, q.cuda(), kd, vd, torch.from_numpy(tables).cuda(),
+                                   torch.from_numpy(lens).cuda(), scale)
+        torch.cuda.synchronize()
+        return out, tables, lens
+
+    before, _, _ = decode()
+    victim = seqs[0]
+    out_ids = pool.swap_out(victim)
+    assert out_ids == model.swap_out(victim)
+    host_k = torch.empty((len(out_ids), Hkv, bs, D), dtype=dtype).pin_memory()
+    host_v = torch.empty_like(host_k).pin_memory()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.swap_blocks(kd, vd, host_k, host_v, torch.tensor(out_ids, dtype=torch.int32, device="cuda"),
+                    to_host=True, err_flag=err)
+    torch.cuda.synchronize()
+    kw, vw = words(k).copy(), words(v).copy()
+    ohk = np.zeros((len(out_ids), Hkv, bs, D), dtype=np.uint16)
+    ohv = np.zeros_like(ohk)
+    oracle.swap_blocks(kw, vw, ohk, ohv, out_ids, to_host=True)
+    assert np.array_equal(words(host_k), ohk) and np.array_equal(words(host_v), ohv)
+    # another sequence takes the freed blocks and overwrites them
+    other, mo = pool.new_seq(), model.new_seq()
+    slots, _ = pool.reserve(other, 200)
+    model.reserve(mo, 200)
+    junk = normal_tensor(rng, (200, Hkv, D), dtype)
+    pkv.paged_kv_append(kd, vd, junk.cuda(), junk.cuda(), torch.from_numpy(slots).cuda())
+    oracle.append(kw, vw, junk, junk, slots)
+    pool.free_seq(other)
+    model.free_seq(mo)
+    in_ids = pool.swap_in(victim)
+    assert in_ids == model.swap_in(victim)
+    pkv.swap_blocks(kd, vd, host_k, host_v, torch.tensor(in_ids, dtype=torch.int32, device="cuda"),
+                    to_host=False, err_flag=err)
+    oracle.swap_blocks(kw, vw, ohk, ohv, in_ids, to_host=False)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert np.array_equal(words(kd.cpu()), kw) and np.array_equal(words(vd.cpu()), vw)
+    after, tables, lens = decode()
+    assert torch.equal(before, after)
+    k_after = torch.from_numpy(kw.view(np.int16)).view(dtype).reshape(k.shape)
+    v_after = torch.from_numpy(vw.view(np.int16)).view(dtype).reshape(v.shape)
+    compare(after, oracle.paged_decode(q, k_after, v_after, tables, lens, scale), what="after swap")
+
+
+def test_swap_blocks_refuses_pageable_host_memory():
+    k, v, _ = _pool(13, 4, 2, 16, 64, torch.float16)
+    kd, vd = k.cuda(), v.cuda()
+    pageable = np.zeros((1, 2, 16, 64), dtype=np.uint16)
+    desc = pkv.cache_desc(kd)
+    ids = torch.tensor([1], dtype=torch.int32, device="cuda")
+    status = _lib.load().swap_blocks(
+        ctypes.byref(desc), ctypes.c_void_p(kd.data_ptr()), ctypes.c_void_p(vd.data_ptr()),
+        pageable.ctypes.data_as(ctypes.c_void_p), pageable.ctypes.data_as(ctypes.c_void_p),
+        ctypes.c_void_p(ids.data_ptr()), 1, 1, None, None)
+    assert status == 1
+    torch.cuda.synchronize()

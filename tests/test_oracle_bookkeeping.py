@@ -41,6 +41,48 @@ def test_golden_exhaustion_trace():
     assert play("pool_exhaustion.txt", _model, PoolExhausted) > 10
 
 
+def test_golden_swap_trace():
+    assert play("swap_trace.txt", _model, PoolExhausted) > 20
+
+
+def test_swap_round_trip_keeps_length_and_conserves_the_pool():
+    """A preempted sequence gives every block back; restoring it takes exactly
+    ceil(len / bs) fresh blocks and it can grow again afterwards."""
+    pool = BlockPoolModel(20, 4, np.random.default_rng(1).permutation(20))
+    a, b = pool.new_seq(), pool.new_seq()
+    pool.reserve(a, 13)
+    pool.reserve(b, 5)
+    shared = pool.fork(a)                          # a's blocks are shared with `shared`
+    free_before = len(pool.free)
+    out = pool.swap_out(a)
+    assert out == pool.table(shared)               # a held the same blocks
+    assert len(pool.free) == free_before           # still held by `shared`
+    pool.free_seq(shared)
+    assert len(pool.free) == free_before + 4
+    _check_invariants_with_swaps(pool)
+    back = pool.swap_in(a)
+    assert len(back) == 4 and pool.length(a) == 13 and all(pool.refcount[x] == 1 for x in back)
+    slots, pairs = pool.reserve(a, 4)
+    assert pairs == [] and len(pool.table(a)) == math.ceil(17 / 4)
+    _check_invariants_with_swaps(pool)
+    with pytest.raises(ValueError):
+        pool.swap_in(a)                            # not swapped
+    pool.swap_out(b)
+    with pytest.raises(ValueError):
+        pool.reserve(b, 1)                         # swapped sequences cannot grow
+
+
+def _check_invariants_with_swaps(pool):
+    in_use = set()
+    for s in pool.seqs.values():
+        if s["swapped"]:
+            assert s["blocks"] == []
+        else:
+            assert len(s["blocks"]) == math.ceil(s["len"] / pool.block_size)
+        in_use.update(s["blocks"])
+    assert len(pool.free) + len(in_use) == pool.num_blocks
+
+
 @pytest.mark.parametrize("bs", [1, 4, 16])
 def test_fresh_block_exactly_when_last_is_full(bs):
     pool = BlockPoolModel(64, bs)

@@ -49,6 +49,10 @@ MUTANTS = {
                          "               sizeof(uint16_t) * (size_t)block_words);", ""),
     "copy direction reversed": ("memcpy(k_cache + dst * block_words, k_cache + src * block_words,",
                                 "memcpy(k_cache + src * block_words, k_cache + dst * block_words,"),
+    "swap uses the list position as the block": ("uint16_t* pk = k_cache + blk * block_words;",
+                                                 "uint16_t* pk = k_cache + i * block_words;"),
+    "swap direction inverted": ("        if (to_host) {\n            memcpy(hk, pk,",
+                                "        if (!to_host) {\n            memcpy(hk, pk,"),
 }
 
 

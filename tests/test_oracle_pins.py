@@ -224,3 +224,25 @@ def test_bad_table_entry_is_reported():
     bad[0, 1] = k.shape[0]
     with pytest.raises(ValueError):
         oracle.paged_decode(q, k, v, bad, lens, 0.3)
+
+
+def test_swap_round_trip_and_relation_to_copy_blocks():
+    """Swapping blocks out and back into other blocks moves their bytes exactly as
+    copy_blocks does; every other block is untouched."""
+    rng = np.random.default_rng(42)
+    NB, Hkv, bs, D = 9, 2, 4, 8
+    k, v = _pool(rng, NB, Hkv, bs, D, torch.bfloat16)
+    kw, vw = oracle.words(k).copy(), oracle.words(v).copy()
+    k0, v0 = kw.copy(), vw.copy()
+    out_ids, in_ids = [2, 7, 0], [5, 1, 8]
+    hk = np.zeros((3, Hkv, bs, D), dtype=np.uint16)
+    hv = np.zeros_like(hk)
+    oracle.swap_blocks(kw, vw, hk, hv, out_ids, to_host=True)
+    assert np.array_equal(kw, k0) and np.array_equal(vw, v0)          # reading changes nothing
+    assert np.array_equal(hk, k0[out_ids]) and np.array_equal(hv, v0[out_ids])
+    oracle.swap_blocks(kw, vw, hk, hv, in_ids, to_host=False)
+    ck, cv = k0.copy(), v0.copy()
+    oracle.copy_blocks(ck, cv, np.array(list(zip(out_ids, in_ids)), dtype=np.int32))
+    assert np.array_equal(kw, ck) and np.array_equal(vw, cv)
+    with pytest.raises(ValueError):
+        oracle.swap_blocks(kw, vw, hk, hv, [NB], to_host=True)

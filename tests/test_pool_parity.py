@@ -15,7 +15,7 @@ def _lib_pool(nb, bs, order):
     return Pool(nb, bs, order)
 
 
-@pytest.mark.parametrize("trace", ["bookkeeping_trace.txt", "pool_exhaustion.txt"])
+@pytest.mark.parametrize("trace", ["bookkeeping_trace.txt", "pool_exhaustion.txt", "swap_trace.txt"])
 def test_golden_traces_on_the_library(trace):
     assert play(trace, _lib_pool, PoolExhausted) > 10
 
@@ -24,7 +24,7 @@ def _same(model, pool, live):
     assert pool.free_list() == model.free_list()
     assert pool.stats() == {k: v for k, v in model.stats().items()} | {}
     for sid in live:
-        assert pool.table(sid) == model.table(sid)
+        assert pool.table(sid) == model.table(sid)  # empty while swapped out
         assert pool.length(sid) == model.length(sid)
     for b in range(model.num_blocks):
         assert pool.refcount(b) == model.refcount[b]
@@ -45,11 +45,15 @@ def test_random_operation_sequences_match_the_model(seed):
             live.append(a)
         elif r < 0.22:
             parent = int(rng.choice(live))
+            if model.seqs[parent]["swapped"]:
+                continue
             a, b = model.fork(parent), pool.fork(parent)
             assert a == b
             live.append(a)
         elif r < 0.75:
             sid, n = int(rng.choice(live)), int(rng.integers(0, 2 * bs + 2))
+            if model.seqs[sid]["swapped"]:
+                continue
             try:
                 ms, mp = model.reserve(sid, n)
             except ModelExhausted:
@@ -58,8 +62,22 @@ def test_random_operation_sequences_match_the_model(seed):
             else:
                 ls, lp = pool.reserve(sid, n)
                 assert list(ls) == ms and lp == [tuple(p) for p in mp]
-        elif r < 0.82:
+        elif r < 0.86:
             sid = int(rng.choice(live))
+            if model.seqs[sid]["swapped"]:
+                try:
+                    mb = model.swap_in(sid)
+                except ModelExhausted:
+                    with pytest.raises(PoolExhausted):
+                        pool.swap_in(sid)
+                else:
+                    assert pool.swap_in(sid) == mb
+            else:
+                assert pool.swap_out(sid) == model.swap_out(sid)
+        elif r < 0.9:
+            sid = int(rng.choice(live))
+            if model.seqs[sid]["swapped"]:
+                continue
             nblk = len(model.table(sid))
             if nblk:
                 i = int(rng.integers(0, nblk))

@@ -1,8 +1,8 @@
 """Replays a golden block-manager trace (tests/golden/*.txt) against a pool object.
 
 The pool object needs: new_seq(), fork(sid), reserve(sid, n) -> (slots, pairs),
-cow(sid, i), free_seq(sid), table(sid), refcount(block) or .refcount[block],
-free_list(), stats() -> dict.  ``exhausted`` is the exception type the pool
+cow(sid, i), free_seq(sid), swap_out(sid) -> blocks, swap_in(sid) -> blocks,
+table(sid), refcount(block) or .refcount[block], free_list(), stats() -> dict.  ``exhausted`` is the exception type the pool
 raises when the free pool cannot cover a request.
 """
 
@@ -63,6 +63,20 @@ def play(name, factory, exhausted):
             pair = pool.cow(int(words[1]), int(words[2]))
             assert (None if pair is None else tuple(pair)) == \
                 (None if rhs == "-" else _pairs(rhs)[0]), line
+        elif op in ("swap_out", "swap_in"):
+            sid = int(words[1])
+            fn = getattr(pool, op)
+            if rhs == "exhausted":
+                before = (pool.table(sid), pool.free_list(), pool.stats())
+                try:
+                    fn(sid)
+                except exhausted:
+                    pass
+                else:
+                    raise AssertionError(f"expected exhaustion: {line}")
+                assert (pool.table(sid), pool.free_list(), pool.stats()) == before, line
+            else:
+                assert list(fn(sid)) == _ints(rhs), line
         elif op == "table":
             assert list(pool.table(int(words[1]))) == _ints(rhs), line
         elif op == "refcount":
