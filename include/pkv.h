@@ -247,6 +247,7 @@ typedef struct pkv_stats {
     int64_t shared_blocks;   /* blocks with reference count > 1                      */
     int64_t num_seqs;        /* resident (not swapped-out) sequences                 */
     int64_t swapped_seqs;    /* swapped-out sequences                                */
+    int64_t cached_blocks;   /* blocks findable by pkv_seq_new_cached                */
 } pkv_stats;
 
 /* free_order: host int32 [num_blocks], a permutation of 0..num_blocks-1, or NULL. */
@@ -270,6 +271,31 @@ pkv_status pkv_seq_fork(pkv_pool* pool, int32_t parent, int32_t* child);
  */
 pkv_status pkv_seq_reserve(pkv_pool* pool, int32_t seq, int32_t n_tokens, int64_t* slots_out,
                            int32_t* cow_pair_out, int32_t* n_cow_out);
+
+/*
+ * Prefix caching ([glossary], paragraph on prefix caching: requests whose
+ * prompts start the same point their block tables at the KV blocks already
+ * computed for that start; [ops page] When to use it: a large system prompt
+ * shared by many requests).  A full block is named by
+ * (the previous block
+ * of its sequence, or -1 for the first block; its block_size token ids).
+ * pkv_seq_reserve_tokens: pkv_seq_reserve for the token ids `tokens` [n_tokens]
+ *   (host int32); every block it fills is registered under its name if its
+ *   predecessor is registered (or it is the first block) and the name is free.
+ *   A sequence grown by pkv_seq_reserve (ids unknown) registers nothing more.
+ * pkv_seq_new_cached: a new sequence that starts on the longest run of
+ *   registered blocks matching the prompt's full blocks, each shared (refcount
+ *   + 1); *n_cached = the tokens covered (a multiple of block_size).  The caller
+ *   appends the rest with pkv_seq_reserve_tokens.
+ * An entry lives while its block is in use: when a block's count reaches 0 its
+ * entry is dropped, with every entry chained below it.  Copies made on write and
+ * blocks returned by swap-in are not registered.
+ */
+pkv_status pkv_seq_reserve_tokens(pkv_pool* pool, int32_t seq, const int32_t* tokens,
+                                  int32_t n_tokens, int64_t* slots_out, int32_t* cow_pair_out,
+                                  int32_t* n_cow_out);
+pkv_status pkv_seq_new_cached(pkv_pool* pool, const int32_t* prompt, int32_t n, int32_t* seq_id,
+                              int32_t* n_cached);
 
 /*
  * Give `seq` a private copy of its logical block `logical_block` if that block

@@ -44,6 +44,26 @@ memory, then restores them later):
   all or nothing, and returns them in logical order (the caller copies the saved
   contents back into them); sharing is not restored: every block comes back
   private.
+
+Prefix caching ("PagedAttention" glossary: the block table enables prefix
+caching, where shared prompt prefixes across requests reuse already-computed KV
+pages; ops page, Example: the shared system prompt is stored once and referenced
+by every session's block table).  Readings:
+
+* a full block's content is named by (the previous block of its sequence, or -1
+  for the first block; the block's token ids), so a lookup walks the chain from
+  the first block and a hit is exact -- no hashing;
+* ``reserve_tokens(seq, tokens)`` is ``reserve`` that also records the token
+  ids; when it fills a block whose predecessor is registered (or that is the
+  sequence's first block), the block is registered unless that name is taken;
+* ``new_cached(prompt)`` starts a sequence on the longest run of registered full
+  blocks matching the prompt's full blocks (each shared, refcount + 1) and
+  returns how many tokens that covers; a sequence whose token ids are unknown
+  (created by ``new_seq`` and grown by ``reserve``) registers nothing;
+* an entry lives only while its block is in use: when a block's count drops to
+  0 (free, swap out, copy on write) its entry is dropped, and so is every entry
+  chained below it (depth first, in registration order); blocks that come back
+  by swap-in are not registered.
 """
 
 from __future__ import annotations
@@ -65,14 +85,17 @@ class BlockPoolModel:
         # The stack's top is the end of the list.
         self.free = list(reversed(order))
         self.refcount = [0] * self.num_blocks
-        self.seqs = {}  # id -> {"blocks": [phys ids], "len": tokens}
+        self.seqs = {}  # id -> {"blocks": [phys ids], "len": tokens, "swapped", "tokens"}
         self.next_id = 0
+        self.cache = {}                     # (previous block or -1, token tuple) -> block
+        self.key_of = {}                    # block -> its name in the cache
+        self.children = {}                  # block -> names registered below it, in order
 
     # -- sequences -----------------------------------------------------------
     def new_seq(self) -> int:
         sid = self.next_id
         self.next_id += 1
-        self.seqs[sid] = {"blocks": [], "len": 0, "swapped": False}
+        self.seqs[sid] = {"blocks": [], "len": 0, "swapped": False, "tokens": None}
         return sid
 
     def _resident(self, sid):
@@ -87,6 +110,7 @@ class BlockPoolModel:
         sid = self.new_seq()
         self.seqs[sid]["blocks"] = list(src["blocks"])
         self.seqs[sid]["len"] = src["len"]
+        self.seqs[sid]["tokens"] = None if src["tokens"] is None else list(src["tokens"])
         for b in src["blocks"]:
             self.refcount[b] += 1
         return sid
@@ -98,6 +122,78 @@ class BlockPoolModel:
 
     def reserve(self, sid: int, n_tokens: int):
         """Make room for ``n_tokens`` more tokens; return (slots, cow_pairs)."""
+        seq = self._resident(sid)
+        out = self._reserve(sid, n_tokens)      # all or nothing
+        if n_tokens:
+            seq["tokens"] = None                # token ids unknown from here on
+        return out
+
+    def reserve_tokens(self, sid: int, tokens):
+        """``reserve`` for these token ids, registering every block it fills."""
+        seq = self._resident(sid)
+        known = seq["tokens"] is not None or seq["len"] == 0
+        slots, pairs = self._reserve(sid, len(tokens))
+        if not known:
+            return slots, pairs
+        if seq["tokens"] is None:
+            seq["tokens"] = []
+        start = len(seq["tokens"])
+        seq["tokens"].extend(int(t) for t in tokens)
+        bs = self.block_size
+        # blocks that became full with this call, in logical order
+        for i in range(start // bs, seq["len"] // bs):
+            if (i + 1) * bs <= start:
+                continue
+            self._register(seq, i)
+        return slots, pairs
+
+    def _register(self, seq, i):
+        blk = seq["blocks"][i]
+        if blk in self.key_of:
+            return
+        prev = -1 if i == 0 else seq["blocks"][i - 1]
+        if i > 0 and prev not in self.key_of:
+            return
+        key = (prev, tuple(seq["tokens"][i * self.block_size:(i + 1) * self.block_size]))
+        if key in self.cache:
+            return
+        self.cache[key] = blk
+        self.key_of[blk] = key
+        if prev >= 0:
+            self.children.setdefault(prev, []).append(key)
+
+    def _drop(self, blk):
+        key = self.key_of.pop(blk, None)
+        if key is None:
+            return
+        del self.cache[key]
+        if key[0] >= 0 and key in self.children.get(key[0], []):
+            self.children[key[0]].remove(key)
+        for child_key in list(self.children.pop(blk, [])):
+            child = self.cache.get(child_key)
+            if child is not None:
+                self._drop(child)
+
+    def new_cached(self, prompt):
+        """A new sequence on the longest cached run of the prompt's full blocks;
+        returns (sequence id, tokens covered)."""
+        sid = self.new_seq()
+        seq = self.seqs[sid]
+        seq["tokens"] = []
+        bs, prev = self.block_size, -1
+        for i in range(len(prompt) // bs):
+            chunk = tuple(int(t) for t in prompt[i * bs:(i + 1) * bs])
+            blk = self.cache.get((prev, chunk))
+            if blk is None:
+                break
+            self.refcount[blk] += 1
+            seq["blocks"].append(blk)
+            seq["tokens"].extend(chunk)
+            prev = blk
+        seq["len"] = len(seq["blocks"]) * bs
+        return sid, seq["len"]
+
+    def _reserve(self, sid: int, n_tokens: int):
         seq = self._resident(sid)
         bs = self.block_size
         length = seq["len"]
@@ -126,7 +222,7 @@ class BlockPoolModel:
                 if self.refcount[cur] > 1:
                     # Writing into a shared block: copy it first.
                     fresh = self._pop()
-                    self.refcount[cur] -= 1
+                    self._decrement(cur)
                     seq["blocks"][pos // bs] = fresh
                     pairs.append((cur, fresh))
             slots.append(seq["blocks"][pos // bs] * bs + pos % bs)
@@ -142,15 +238,20 @@ class BlockPoolModel:
         if not self.free:
             raise PoolExhausted("no free block for the copy")
         fresh = self._pop()
-        self.refcount[cur] -= 1
-        seq["blocks"][logical_block] = fresh
+        self._decrement(cur)
+        seq["blocks"][logical_block] = fresh  # the copy is not registered
         return (cur, fresh)
+
+    def _decrement(self, b) -> None:
+        """refcount - 1; at 0 the block leaves the cache and goes to the free pool."""
+        self.refcount[b] -= 1
+        if self.refcount[b] == 0:
+            self._drop(b)
+            self.free.append(b)
 
     def _release(self, blocks) -> None:
         for b in blocks:
-            self.refcount[b] -= 1
-            if self.refcount[b] == 0:
-                self.free.append(b)
+            self._decrement(b)
 
     def free_seq(self, sid: int) -> None:
         seq = self.seqs.pop(sid)
@@ -204,6 +305,7 @@ class BlockPoolModel:
             "shared_blocks": sum(1 for r in self.refcount if r > 1),
             "num_seqs": len(resident),
             "swapped_seqs": len(self.seqs) - len(resident),
+            "cached_blocks": len(self.cache),
         }
 
 

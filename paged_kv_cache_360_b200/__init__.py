@@ -219,6 +219,29 @@ class Pool:
                                              pair.ctypes.data_as(ctypes.c_void_p), ctypes.byref(n)))
         return slots[:n_tokens], ([(int(pair[0]), int(pair[1]))] if n.value else [])
 
+    def reserve_tokens(self, seq: int, tokens):
+        """reserve() for these token ids, registering the blocks it fills in the
+        prefix cache; returns (slots, [(src, dst)] copy pairs)."""
+        toks = np.ascontiguousarray(tokens, dtype=np.int32)
+        n_tokens = len(toks)
+        slots = np.empty(max(1, n_tokens), dtype=np.int64)
+        pair = np.empty(2, dtype=np.int32)
+        n = ctypes.c_int32()
+        _lib.check(self._lib.pkv_seq_reserve_tokens(
+            self._h, seq, toks.ctypes.data_as(ctypes.c_void_p), n_tokens,
+            slots.ctypes.data_as(ctypes.c_void_p), pair.ctypes.data_as(ctypes.c_void_p),
+            ctypes.byref(n)))
+        return slots[:n_tokens], ([(int(pair[0]), int(pair[1]))] if n.value else [])
+
+    def new_cached(self, prompt):
+        """A new sequence on the longest cached prefix of `prompt`;
+        returns (sequence id, tokens covered)."""
+        toks = np.ascontiguousarray(prompt, dtype=np.int32)
+        sid, covered = ctypes.c_int32(), ctypes.c_int32()
+        _lib.check(self._lib.pkv_seq_new_cached(self._h, toks.ctypes.data_as(ctypes.c_void_p),
+                                                len(toks), ctypes.byref(sid), ctypes.byref(covered)))
+        return sid.value, covered.value
+
     def cow(self, seq: int, logical_block: int):
         pair = np.empty(2, dtype=np.int32)
         n = ctypes.c_int32()

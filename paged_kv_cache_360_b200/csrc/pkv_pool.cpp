@@ -10,8 +10,10 @@
 // caller-given order, logical-order release, ids counting up, all-or-nothing
 // requests) are stated in pkv.h.
 #include <cstdint>
+#include <map>
 #include <new>
 #include <unordered_set>
+#include <utility>
 #include <vector>
 
 #include "pkv.h"
@@ -24,11 +26,59 @@ struct pkv_pool {
     std::vector<int32_t> refcount;
     struct Seq {
         bool live = false;
-        bool swapped = false;  // preempted: blocks given back, length kept
+        bool swapped = false;       // preempted: blocks given back, length kept
+        bool tokens_known = false;  // `tokens` holds every token id of the sequence
         int64_t len = 0;
         std::vector<int32_t> blocks;
+        std::vector<int32_t> tokens;
     };
     std::vector<Seq> seqs;  // index = sequence id
+
+    // Prefix cache: a full block is named by (previous block or -1, its token
+    // ids).  An entry lives while its block is in use.
+    using Key = std::pair<int32_t, std::vector<int32_t>>;
+    std::map<Key, int32_t> cache;
+    std::vector<char> registered;            // per block
+    std::vector<Key> key_of;                 // per block, valid when registered
+    std::vector<std::vector<Key>> children;  // per block: names registered below it, in order
+
+    // Drop a block's entry and, depth first, every entry chained below it.
+    void drop(int32_t b) {
+        if (!registered[b]) return;
+        registered[b] = 0;
+        const Key key = key_of[b];
+        cache.erase(key);
+        if (key.first >= 0) {
+            auto& sib = children[key.first];
+            for (size_t i = 0; i < sib.size(); ++i)
+                if (sib[i] == key) {
+                    sib.erase(sib.begin() + static_cast<std::ptrdiff_t>(i));
+                    break;
+                }
+        }
+        std::vector<Key> below = std::move(children[b]);
+        children[b].clear();
+        for (const Key& k : below) {
+            auto it = cache.find(k);
+            if (it != cache.end()) drop(it->second);
+        }
+    }
+
+    // Register logical block i of `s` (full, token ids known) unless its block is
+    // already named, its predecessor is not registered, or the name is taken.
+    void register_block(const Seq& s, int64_t i) {
+        const int32_t b = s.blocks[i];
+        if (registered[b]) return;
+        const int32_t prev = i == 0 ? -1 : s.blocks[i - 1];
+        if (i > 0 && !registered[prev]) return;
+        Key key(prev, std::vector<int32_t>(s.tokens.begin() + i * block_size,
+                                           s.tokens.begin() + (i + 1) * block_size));
+        if (cache.count(key)) return;
+        cache.emplace(key, b);
+        registered[b] = 1;
+        key_of[b] = key;
+        if (prev >= 0) children[prev].push_back(std::move(key));
+    }
 
     Seq* find(int32_t id) {
         if (id < 0 || id >= static_cast<int32_t>(seqs.size()) || !seqs[id].live) return nullptr;
@@ -48,10 +98,16 @@ struct pkv_pool {
         Seq* s = find(id);
         return (s && !s->swapped) ? s : nullptr;
     }
-    // refcount - 1 per block, logical order; blocks reaching 0 go on the free stack
+    // refcount - 1; at 0 the block leaves the cache and goes on the free stack
+    void decrement(int32_t b) {
+        if (--refcount[b] == 0) {
+            drop(b);
+            free_stack.push_back(b);
+        }
+    }
+    // decrement every block, logical order
     void release(const std::vector<int32_t>& blocks) {
-        for (int32_t b : blocks)
-            if (--refcount[b] == 0) free_stack.push_back(b);
+        for (int32_t b : blocks) decrement(b);
     }
 };
 
@@ -68,6 +124,9 @@ extern "C" pkv_status pkv_pool_create(int32_t num_blocks, int32_t block_size,
     p->num_blocks = num_blocks;
     p->block_size = block_size;
     p->refcount.assign(num_blocks, 0);
+    p->registered.assign(num_blocks, 0);
+    p->key_of.resize(num_blocks);
+    p->children.resize(num_blocks);
     p->free_stack.resize(num_blocks);
     if (free_order) {
         std::vector<char> seen(num_blocks, 0);
@@ -109,13 +168,10 @@ extern "C" pkv_status pkv_seq_fork(pkv_pool* pool, int32_t parent, int32_t* chil
     return PKV_OK;
 }
 
-extern "C" pkv_status pkv_seq_reserve(pkv_pool* pool, int32_t seq, int32_t n_tokens,
-                                      int64_t* slots_out, int32_t* cow_pair_out,
-                                      int32_t* n_cow_out) {
-    if (!pool || n_tokens < 0 || (n_tokens > 0 && !slots_out))
-        return fail(PKV_ERR_INVALID_ARG, "pkv_seq_reserve: bad argument");
-    pkv_pool::Seq* s = pool->resident(seq);
-    if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_reserve: unknown or swapped-out sequence");
+namespace {
+
+pkv_status reserve_impl(pkv_pool* pool, pkv_pool::Seq* s, int32_t n_tokens, int64_t* slots_out,
+                        int32_t* cow_pair_out, int32_t* n_cow_out) {
     const int64_t bs = pool->block_size;
     if (n_cow_out) *n_cow_out = 0;
     // Blocks needed: one per block boundary crossed, plus a copy if the first
@@ -137,7 +193,7 @@ extern "C" pkv_status pkv_seq_reserve(pkv_pool* pool, int32_t seq, int32_t n_tok
         const int64_t i = s->len / bs;
         const int32_t src = s->blocks[i];
         const int32_t dst = pool->pop();
-        pool->refcount[src] -= 1;
+        pool->decrement(src);
         s->blocks[i] = dst;
         cow_pair_out[0] = src;
         cow_pair_out[1] = dst;
@@ -149,6 +205,68 @@ extern "C" pkv_status pkv_seq_reserve(pkv_pool* pool, int32_t seq, int32_t n_tok
         slots_out[k] = static_cast<int64_t>(s->blocks[pos / bs]) * bs + pos % bs;
         s->len = pos + 1;
     }
+    return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" pkv_status pkv_seq_reserve(pkv_pool* pool, int32_t seq, int32_t n_tokens,
+                                      int64_t* slots_out, int32_t* cow_pair_out,
+                                      int32_t* n_cow_out) {
+    if (!pool || n_tokens < 0 || (n_tokens > 0 && !slots_out))
+        return fail(PKV_ERR_INVALID_ARG, "pkv_seq_reserve: bad argument");
+    pkv_pool::Seq* s = pool->resident(seq);
+    if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_reserve: unknown or swapped-out sequence");
+    const pkv_status st = reserve_impl(pool, s, n_tokens, slots_out, cow_pair_out, n_cow_out);
+    if (st == PKV_OK && n_tokens > 0) {  // the token ids are unknown from here on
+        s->tokens_known = false;
+        s->tokens.clear();
+    }
+    return st;
+}
+
+extern "C" pkv_status pkv_seq_reserve_tokens(pkv_pool* pool, int32_t seq, const int32_t* tokens,
+                                             int32_t n_tokens, int64_t* slots_out,
+                                             int32_t* cow_pair_out, int32_t* n_cow_out) {
+    if (!pool || n_tokens < 0 || (n_tokens > 0 && (!slots_out || !tokens)))
+        return fail(PKV_ERR_INVALID_ARG, "pkv_seq_reserve_tokens: bad argument");
+    pkv_pool::Seq* s = pool->resident(seq);
+    if (!s) return fail(PKV_ERR_INVALID_ARG, "pkv_seq_reserve_tokens: unknown or swapped-out sequence");
+    const bool known = s->tokens_known || s->len == 0;
+    const pkv_status st = reserve_impl(pool, s, n_tokens, slots_out, cow_pair_out, n_cow_out);
+    if (st != PKV_OK || !known) return st;
+    s->tokens_known = true;
+    const int64_t start = static_cast<int64_t>(s->tokens.size());
+    s->tokens.insert(s->tokens.end(), tokens, tokens + n_tokens);
+    const int64_t bs = pool->block_size;
+    for (int64_t i = start / bs; i < s->len / bs; ++i)
+        if ((i + 1) * bs > start) pool->register_block(*s, i);
+    return PKV_OK;
+}
+
+extern "C" pkv_status pkv_seq_new_cached(pkv_pool* pool, const int32_t* prompt, int32_t n,
+                                         int32_t* seq_id, int32_t* n_cached) {
+    if (!pool || !seq_id || !n_cached || n < 0 || (n > 0 && !prompt))
+        return fail(PKV_ERR_INVALID_ARG, "pkv_seq_new_cached: bad argument");
+    pool->seqs.emplace_back();
+    pkv_pool::Seq& s = pool->seqs.back();
+    s.live = true;
+    s.tokens_known = true;
+    const int32_t bs = pool->block_size;
+    int32_t prev = -1;
+    for (int32_t i = 0; i < n / bs; ++i) {
+        pkv_pool::Key key(prev, std::vector<int32_t>(prompt + i * bs, prompt + (i + 1) * bs));
+        auto it = pool->cache.find(key);
+        if (it == pool->cache.end()) break;
+        const int32_t b = it->second;
+        pool->refcount[b] += 1;
+        s.blocks.push_back(b);
+        s.tokens.insert(s.tokens.end(), key.second.begin(), key.second.end());
+        prev = b;
+    }
+    s.len = static_cast<int64_t>(s.blocks.size()) * bs;
+    *seq_id = static_cast<int32_t>(pool->seqs.size() - 1);
+    *n_cached = static_cast<int32_t>(s.len);
     return PKV_OK;
 }
 
@@ -165,8 +283,8 @@ extern "C" pkv_status pkv_seq_cow(pkv_pool* pool, int32_t seq, int32_t logical_b
     if (pool->free_stack.empty())
         return fail(PKV_ERR_NO_FREE_BLOCK, "pkv_seq_cow: free pool exhausted");
     const int32_t dst = pool->pop();
-    pool->refcount[src] -= 1;
-    s->blocks[logical_block] = dst;
+    pool->decrement(src);
+    s->blocks[logical_block] = dst;  // the copy is not registered
     pair_out[0] = src;
     pair_out[1] = dst;
     *n_out = 1;
@@ -180,9 +298,12 @@ extern "C" pkv_status pkv_seq_free(pkv_pool* pool, int32_t seq) {
     pool->release(s->blocks);
     s->blocks.clear();
     s->blocks.shrink_to_fit();
+    s->tokens.clear();
+    s->tokens.shrink_to_fit();
     s->len = 0;
     s->live = false;
     s->swapped = false;
+    s->tokens_known = false;
     return PKV_OK;
 }
 
@@ -303,5 +424,6 @@ extern "C" pkv_status pkv_pool_stats(const pkv_pool* pool, pkv_stats* st) {
     st->live_slots = static_cast<int64_t>(live.size());
     st->shared_blocks = 0;
     for (int32_t r : pool->refcount) st->shared_blocks += r > 1;
+    st->cached_blocks = static_cast<int64_t>(pool->cache.size());
     return PKV_OK;
 }

@@ -479,3 +479,75 @@ def test_swap_blocks_refuses_pageable_host_memory():
         ctypes.c_void_p(ids.data_ptr()), 1, 1, None, None)
     assert status == 1
     torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------ prefix caching
+
+def _prefix_rows(tokens, Hkv, D, dtype):
+    """K and V rows [len, Hkv, D] where the row at position p depends only on
+    tokens[:p + 1] -- as a model's keys and values do, so that requests with the
+    same prompt prefix have the same rows there."""
+    ks, vs = [], []
+    for p in range(len(tokens)):
+        rng = np.random.default_rng([7] + [int(t) for t in tokens[:p + 1]])
+        ks.append(normal_tensor(rng, (Hkv, D), dtype))
+        vs.append(normal_tensor(rng, (Hkv, D), dtype))
+    return torch.stack(ks), torch.stack(vs)
+
+
+@pytest.mark.parametrize("dtype,D,bs", [(torch.bfloat16, 128, 16), (torch.float16, 64, 32)])
+def test_prefix_cached_requests_share_blocks_and_decode_correctly(dtype, D, bs):
+    """Three requests with a common system prompt: the second and third start on
+    the first one's full prompt blocks (shared, not recomputed), append only
+    their own tokens, and decode to the dense oracle over their whole, unpaged
+    token rows; the pool matches the oracle's pool after the same appends."""
+    rng = np.random.default_rng(21)
+    Hkv, H, NB = 2, 8, 48
+    system = list(rng.integers(0, 1000, size=3 * bs - 5))
+    prompts = [system + list(rng.integers(0, 1000, size=n)) for n in (bs + 3, 2 * bs, 7)]
+    pool = pkv.Pool(NB, bs, rng.permutation(NB))
+    model = oracle.BlockPoolModel(NB, bs, pool.free_list())
+    k0, v0, _ = _pool(22, NB, Hkv, bs, D, dtype)      # stale contents everywhere
+    kd, vd = k0.cuda(), v0.cuda()
+    kw, vw = words(k0).copy(), words(v0).copy()
+    seqs, covered = [], []
+    for prompt in prompts:
+        sid, n = pool.new_cached(prompt)
+        assert (sid, n) == model.new_cached(prompt)
+        slots, pairs = pool.reserve_tokens(sid, prompt[n:])
+        assert (list(slots), pairs) == model.reserve_tokens(sid, prompt[n:])
+        assert pairs == []
+        kr, vr = _prefix_rows(prompt, Hkv, D, dtype)
+        pkv.paged_kv_append(kd, vd, kr[n:].cuda(), vr[n:].cuda(), torch.from_numpy(slots).cuda())
+        oracle.append(kw, vw, kr[n:], vr[n:], slots)
+        seqs.append(sid)
+        covered.append(n)
+    # the system prompt's two full blocks are shared by all three requests
+    full = (len(system) // bs) * bs
+    assert covered == [0, full, full]
+    for b in pool.table(seqs[0])[:full // bs]:
+        assert pool.refcount(b) == 3
+    assert pool.stats() == model.stats()
+    torch.cuda.synchronize()
+    assert np.array_equal(words(kd.cpu()), kw) and np.array_equal(words(vd.cpu()), vw)
+
+    q = normal_tensor(rng, (3, H, D), dtype)
+    mb = max(len(pool.table(s)) for s in seqs)
+    tables, lens = pool.block_tables(seqs, mb)
+    out = torch.empty((3, H, D), dtype=dtype, device="cuda")
+    scale = float(np.float32(1.0 / np.sqrt(D)))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.paged_attention_decode(out, q.cuda(), kd, vd, torch.from_numpy(tables).cuda(),
+                               torch.from_numpy(lens).cuda(), scale, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    code = oracle.BF16 if dtype == torch.bfloat16 else oracle.F16
+    ref = np.empty((3, H, D))
+    for i, prompt in enumerate(prompts):
+        kr, vr = _prefix_rows(prompt, Hkv, D, dtype)
+        K, V, Q = oracle.widen(words(kr), code), oracle.widen(words(vr), code), \
+            oracle.widen(words(q[i]), code)
+        for h in range(H):
+            hk = h // (H // Hkv)
+            ref[i, h] = oracle.attend_dense(Q[h], K[:, hk], V[:, hk], scale)
+    compare(out, ref, what="prefix-cached requests")

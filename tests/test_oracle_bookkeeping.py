@@ -45,6 +45,77 @@ def test_golden_swap_trace():
     assert play("swap_trace.txt", _model, PoolExhausted) > 20
 
 
+def test_golden_prefix_cache_trace():
+    assert play("prefix_cache_trace.txt", _model, PoolExhausted) > 20
+
+
+def test_prefix_cache_shares_only_identical_prefixes():
+    """Two prompts share exactly the full blocks of their common prefix; a block
+    is never found under a different prefix."""
+    bs = 4
+    pool = BlockPoolModel(64, bs)
+    a = pool.new_seq()
+    prompt = list(range(100, 123))                 # 23 tokens: 5 full blocks + 3
+    pool.reserve_tokens(a, prompt)
+    assert pool.stats()["cached_blocks"] == 5
+    for n_same in range(0, 23):
+        other = prompt[:n_same] + [7] * (23 - n_same)
+        sid, covered = pool.new_cached(other)
+        assert covered == (n_same // bs) * bs
+        assert pool.table(sid) == pool.table(a)[:n_same // bs]
+        pool.free_seq(sid)
+    # the same block contents after a different first block are not a hit
+    b = pool.new_seq()
+    pool.reserve_tokens(b, [9, 9, 9, 9] + prompt[4:8])
+    sid, covered = pool.new_cached([1, 2, 3, 4] + prompt[4:8])
+    assert covered == 0
+    # dropping a block drops every entry chained below it
+    pool.free_seq(a)
+    assert pool.stats()["cached_blocks"] == 2      # b's two blocks
+    sid, covered = pool.new_cached(prompt)
+    assert covered == 0
+
+
+def test_prefix_cache_random_operations_keep_invariants():
+    rng = np.random.default_rng(9)
+    pool = BlockPoolModel(48, 2, rng.permutation(48))
+    live = []
+    vocab = [1, 2, 3]
+    for _ in range(600):
+        r = rng.random()
+        try:
+            if r < 0.2 or not live:
+                prompt = [int(x) for x in rng.choice(vocab, size=int(rng.integers(0, 9)))]
+                sid, covered = pool.new_cached(prompt)
+                assert covered % 2 == 0 and covered <= len(prompt)
+                live.append(sid)
+                pool.reserve_tokens(sid, prompt[covered:])
+            elif r < 0.6:
+                sid = int(rng.choice(live))
+                if not pool.seqs[sid]["swapped"]:
+                    pool.reserve_tokens(sid, [int(x) for x in rng.choice(vocab, size=int(rng.integers(1, 4)))])
+            elif r < 0.7:
+                sid = int(rng.choice(live))
+                if not pool.seqs[sid]["swapped"]:
+                    live.append(pool.fork(sid))
+            else:
+                sid = int(rng.choice(live))
+                live.remove(sid)
+                pool.free_seq(sid)
+        except PoolExhausted:
+            pass
+        _check_invariants_with_swaps(pool)
+        # every entry names a block in use whose tokens match its name
+        for (prev, toks), blk in pool.cache.items():
+            assert pool.refcount[blk] > 0
+            holders = [s for s in pool.seqs.values() if blk in s["blocks"] and s["tokens"] is not None]
+            for s in holders:
+                i = s["blocks"].index(blk)
+                if len(s["tokens"]) >= (i + 1) * 2:
+                    assert tuple(s["tokens"][2 * i:2 * i + 2]) == toks
+                    assert (s["blocks"][i - 1] if i else -1) == prev
+
+
 def test_swap_round_trip_keeps_length_and_conserves_the_pool():
     """A preempted sequence gives every block back; restoring it takes exactly
     ceil(len / bs) fresh blocks and it can grow again afterwards."""

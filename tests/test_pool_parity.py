@@ -15,19 +15,100 @@ def _lib_pool(nb, bs, order):
     return Pool(nb, bs, order)
 
 
-@pytest.mark.parametrize("trace", ["bookkeeping_trace.txt", "pool_exhaustion.txt", "swap_trace.txt"])
+@pytest.mark.parametrize("trace", ["bookkeeping_trace.txt", "pool_exhaustion.txt", "swap_trace.txt",
+                                   "prefix_cache_trace.txt"])
 def test_golden_traces_on_the_library(trace):
     assert play(trace, _lib_pool, PoolExhausted) > 10
 
 
 def _same(model, pool, live):
     assert pool.free_list() == model.free_list()
-    assert pool.stats() == {k: v for k, v in model.stats().items()} | {}
+    assert pool.stats() == model.stats()
     for sid in live:
         assert pool.table(sid) == model.table(sid)  # empty while swapped out
         assert pool.length(sid) == model.length(sid)
     for b in range(model.num_blocks):
         assert pool.refcount(b) == model.refcount[b]
+
+
+def _reserve_both(model, pool, sid, n, tokens=None):
+    try:
+        ms, mp = model.reserve(sid, n) if tokens is None else model.reserve_tokens(sid, tokens)
+    except ModelExhausted:
+        with pytest.raises(PoolExhausted):
+            pool.reserve(sid, n) if tokens is None else pool.reserve_tokens(sid, tokens)
+    else:
+        ls, lp = pool.reserve(sid, n) if tokens is None else pool.reserve_tokens(sid, tokens)
+        assert list(ls) == ms and lp == [tuple(p) for p in mp]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_prefix_cached_operation_sequences_match_the_model(seed):
+    """Requests built from a few shared prompt stems (so that cache hits, partial
+    hits and misses all happen), grown by token ids or by anonymous tokens,
+    forked, copied on write, swapped and freed in a seeded random order."""
+    rng = np.random.default_rng(900 + seed)
+    nb, bs = int(rng.integers(12, 64)), int(rng.choice([1, 2, 4, 8]))
+    order = rng.permutation(nb)
+    model, pool = BlockPoolModel(nb, bs, order), Pool(nb, bs, order)
+    stems = [list(rng.integers(0, 5, size=int(rng.integers(0, 4 * bs + 3)))) for _ in range(3)]
+    live = []
+    for step in range(400):
+        r = rng.random()
+        if r < 0.2 or not live:
+            prompt = list(stems[int(rng.integers(0, 3))]) + \
+                list(rng.integers(0, 5, size=int(rng.integers(0, 2 * bs + 1))))
+            a, b = model.new_cached(prompt), pool.new_cached(prompt)
+            assert a == b
+            live.append(a[0])
+            _reserve_both(model, pool, a[0], 0, prompt[a[1]:])
+        elif r < 0.3:
+            parent = int(rng.choice(live))
+            if model.seqs[parent]["swapped"]:
+                continue
+            a, b = model.fork(parent), pool.fork(parent)
+            assert a == b
+            live.append(a)
+        elif r < 0.65:
+            sid = int(rng.choice(live))
+            if model.seqs[sid]["swapped"]:
+                continue
+            n = int(rng.integers(0, 2 * bs + 2))
+            anonymous = rng.random() < 0.15
+            _reserve_both(model, pool, sid, n,
+                          None if anonymous else list(rng.integers(0, 5, size=n)))
+        elif r < 0.75:
+            sid = int(rng.choice(live))
+            if model.seqs[sid]["swapped"]:
+                try:
+                    mb = model.swap_in(sid)
+                except ModelExhausted:
+                    with pytest.raises(PoolExhausted):
+                        pool.swap_in(sid)
+                else:
+                    assert pool.swap_in(sid) == mb
+            else:
+                assert pool.swap_out(sid) == model.swap_out(sid)
+        elif r < 0.8:
+            sid = int(rng.choice(live))
+            nblk = len(model.table(sid))
+            if model.seqs[sid]["swapped"] or not nblk:
+                continue
+            i = int(rng.integers(0, nblk))
+            try:
+                mp = model.cow(sid, i)
+            except ModelExhausted:
+                with pytest.raises(PoolExhausted):
+                    pool.cow(sid, i)
+            else:
+                assert pool.cow(sid, i) == mp
+        else:
+            sid = int(rng.choice(live))
+            live.remove(sid)
+            model.free_seq(sid)
+            pool.free_seq(sid)
+        _same(model, pool, live)
+    assert model.stats()["cached_blocks"] >= 0
 
 
 @pytest.mark.parametrize("seed", range(6))

@@ -63,6 +63,17 @@ def play(name, factory, exhausted):
             pair = pool.cow(int(words[1]), int(words[2]))
             assert (None if pair is None else tuple(pair)) == \
                 (None if rhs == "-" else _pairs(rhs)[0]), line
+        elif op == "reserve_tokens":
+            sid, toks = int(words[1]), [int(x) for x in words[2].split(":")]
+            slots, pairs = pool.reserve_tokens(sid, toks)
+            exp = rhs.split()
+            assert list(slots) == _ints(exp[1]), (line, slots)
+            assert [tuple(p) for p in pairs] == _pairs(exp[3]), (line, pairs)
+        elif op == "new_cached":
+            toks = [int(x) for x in words[1].split(":")]
+            sid, covered = pool.new_cached(toks)
+            exp = rhs.split()
+            assert (sid, covered) == (int(exp[0]), int(exp[1])), (line, sid, covered)
         elif op in ("swap_out", "swap_in"):
             sid = int(words[1])
             fn = getattr(pool, op)
