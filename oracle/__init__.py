@@ -64,6 +64,9 @@ def _load():
             lib.oracle_paged_decode_split.restype = ctypes.c_int
             lib.oracle_paged_decode_split.argtypes = [ctypes.c_int, p, p, p, p, i32, p, i32, i32,
                                                       i32, i32, i32, i32, dbl, i32, p]
+            lib.oracle_paged_prefill.restype = ctypes.c_int
+            lib.oracle_paged_prefill.argtypes = [ctypes.c_int, p, p, p, p, i32, p, p, i32, i32,
+                                                 i32, i32, i32, i32, dbl, p]
             lib.oracle_append.restype = ctypes.c_int
             lib.oracle_append.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i32]
             lib.oracle_copy_blocks.restype = ctypes.c_int
@@ -151,6 +154,31 @@ def paged_decode_split(q, k_cache, v_cache, block_tables, context_lens, scale,
                                            float(scale), int(partition_size), _ptr(out))
     if rc != 0:
         raise ValueError(f"oracle_paged_decode_split failed ({rc})")
+    return out
+
+
+def paged_prefill(q, k_cache, v_cache, block_tables, context_lens, query_start, scale) -> np.ndarray:
+    """Causal prefill attention through the block tables; returns float64 [T, H, D].
+
+    q: fp16/bf16 [T, H, D], sequence b's query tokens in rows
+    query_start[b] .. query_start[b+1]-1, the last ones of its context_lens[b]
+    tokens; caches [NB, Hkv, bs, D]; block_tables int32 [B, MB].
+    """
+    dt = dtype_code(q)
+    T, H, D = q.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    qw, kw, vw = _words(q), _words(k_cache), _words(v_cache)
+    tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    qs = np.ascontiguousarray(query_start, dtype=np.int32)
+    B = len(lens)
+    assert len(qs) == B + 1 and qs[-1] == T
+    out = np.zeros((T, H, D), dtype=np.float64)
+    rc = _load().oracle_paged_prefill(dt, _ptr(qw), _ptr(kw), _ptr(vw), _ptr(tables),
+                                      tables.shape[1], _ptr(lens), _ptr(qs), B, H, Hkv, D, bs,
+                                      NB, float(scale), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_paged_prefill failed ({rc})")
     return out
 
 

@@ -33,9 +33,10 @@
  *   - fp16 / bf16 storage values are widened exactly to double.
  *
  * Parity status: every exported function is pinned by tests under tests/
- * (brute force against torch's scaled_dot_product_attention in float64,
- * closed forms, block-permutation invariance, contiguous-slab equality, the
- * split identity, and byte round trips); none is "parity unpinned".
+ * (brute force against torch's scaled_dot_product_attention in float64, with
+ * is_causal for the prefill, closed forms, block-permutation invariance,
+ * contiguous-slab equality, the split identity, chunked-prefill consistency,
+ * and byte round trips); none is "parity unpinned".
  */
 #include <math.h>
 #include <stdint.h>
@@ -257,6 +258,66 @@ int oracle_paged_decode_split(int dtype, const uint16_t* q, const uint16_t* k_ca
         }
     }
     free(K); free(V); free(s); free(qd); free(mp); free(lp); free(op);
+    return rc;
+}
+
+/* ------------------------------------------------------ paged prefill */
+
+/*
+ * Paged prefill, the definition: the prompt phase reads keys and values
+ * through the same block table as decode ([ops page] How it works: the
+ * attention kernel reads KV through the block table; Concept: prompt
+ * processing is the compute-heavy phase).  Sequence b holds context_lens[b]
+ * tokens in the pool, of which the last n_b = query_start[b + 1] -
+ * query_start[b] are this step's query tokens (their keys and values already
+ * appended).  Query token i of sequence b sits at position
+ * p = context_lens[b] - n_b + i and attends causally to tokens 0 .. p.
+ *   q:           [T][H][D] storage words, T = query_start[B], sequence b's
+ *                queries in rows query_start[b] .. query_start[b + 1] - 1
+ *   query_start: int32 [B + 1], non-decreasing, query_start[0] = 0
+ *   out:         double [T][H][D]
+ * n_b = 1 is decode of the last token; n_b = context_lens[b] is a whole prompt.
+ * Returns 0, -1 on a bad table entry, -2 on bad shapes (n_b < 0 or
+ * n_b > context_lens[b], a length past the table), -3 on allocation failure.
+ */
+int oracle_paged_prefill(int dtype, const uint16_t* q, const uint16_t* k_cache,
+                         const uint16_t* v_cache, const int32_t* block_tables,
+                         int32_t max_blocks, const int32_t* context_lens,
+                         const int32_t* query_start, int32_t B, int32_t H, int32_t Hkv,
+                         int32_t D, int32_t block_size, int32_t num_blocks, double scale,
+                         double* out) {
+    if (H <= 0 || Hkv <= 0 || H % Hkv != 0 || D <= 0 || block_size <= 0) return -2;
+    if (query_start[0] != 0) return -2;
+    int32_t group = H / Hkv;
+    int64_t max_len = (int64_t)max_blocks * block_size;
+    double* K = malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1) * D);
+    double* V = malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1) * D);
+    double* s = malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1));
+    double* qd = malloc(sizeof(double) * (size_t)D);
+    int rc = (K && V && s && qd) ? 0 : -3;
+    for (int32_t b = 0; rc == 0 && b < B; ++b) {
+        int64_t L = context_lens[b];
+        int64_t n = (int64_t)query_start[b + 1] - query_start[b];
+        if (L < 0 || L > max_len || n < 0 || n > L) { rc = -2; break; }
+        for (int32_t hk = 0; rc == 0 && hk < Hkv; ++hk) {
+            if (gather_kv(dtype, k_cache, v_cache, block_tables + (int64_t)b * max_blocks,
+                          num_blocks, Hkv, block_size, D, hk, 0, L, K, V) != 0) {
+                rc = -1;
+                break;
+            }
+            for (int64_t i = 0; i < n; ++i) {
+                int64_t row = query_start[b] + i;
+                int64_t p = L - n + i;
+                for (int32_t j = 0; j < group; ++j) {
+                    int32_t h = hk * group + j;
+                    const uint16_t* qrow = q + (row * H + h) * D;
+                    for (int32_t d = 0; d < D; ++d) qd[d] = widen(dtype, qrow[d]);
+                    oracle_attend_dense(qd, K, V, p + 1, D, scale, s, out + (row * H + h) * D);
+                }
+            }
+        }
+    }
+    free(K); free(V); free(s); free(qd);
     return rc;
 }
 

@@ -51,6 +51,14 @@ MUTANTS = {
                                 "memcpy(k_cache + src * block_words, k_cache + dst * block_words,"),
     "swap uses the list position as the block": ("uint16_t* pk = k_cache + blk * block_words;",
                                                  "uint16_t* pk = k_cache + i * block_words;"),
+    "prefill causal bound off by one": ("oracle_attend_dense(qd, K, V, p + 1, D,",
+                                        "oracle_attend_dense(qd, K, V, p, D,"),
+    "prefill sees the whole context": ("oracle_attend_dense(qd, K, V, p + 1, D,",
+                                       "oracle_attend_dense(qd, K, V, L, D,"),
+    "prefill position ignores the context": ("int64_t p = L - n + i;", "int64_t p = i;"),
+    "prefill query row ignores the sequence offset": ("int64_t row = query_start[b] + i;",
+                                                      "int64_t row = i;"),
+    "prefill GQA mapping interleaved": ("int32_t h = hk * group + j;", "int32_t h = hk + j * Hkv;"),
     "swap direction inverted": ("        if (to_host) {\n            memcpy(hk, pk,",
                                 "        if (!to_host) {\n            memcpy(hk, pk,"),
 }

@@ -246,3 +246,86 @@ def test_swap_round_trip_and_relation_to_copy_blocks():
     assert np.array_equal(kw, ck) and np.array_equal(vw, cv)
     with pytest.raises(ValueError):
         oracle.swap_blocks(kw, vw, hk, hv, [NB], to_host=True)
+
+
+# ------------------------------------------------------------ paged prefill
+
+def _prefill_case(seed, lens, nq, H=4, Hkv=2, D=8, bs=4, dtype=torch.bfloat16):
+    """Logical-order pool (as _identity_case) plus nq[b] query tokens per sequence."""
+    q1, k, v, tables, lens, MB = _identity_case(seed, B=len(lens), H=H, Hkv=Hkv, D=D, bs=bs,
+                                                lens=lens, dtype=dtype)
+    rng = np.random.default_rng(seed + 1000)
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    q = torch.from_numpy(rng.standard_normal((int(qs[-1]), H, D), dtype=np.float32)).to(dtype)
+    return q, k, v, tables, lens, MB, qs
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("H,Hkv", [(4, 4), (8, 2)])
+def test_prefill_whole_prompt_matches_sdpa_is_causal(dtype, H, Hkv):
+    """A whole prompt (queries = every context token) is torch's causal SDPA,
+    is_causal=True, over the logical slab, in float64."""
+    lens = (37, 9, 1)
+    q, k, v, tables, lens, MB, qs = _prefill_case(40 + H, lens, lens, H=H, Hkv=Hkv, dtype=dtype)
+    out = oracle.paged_prefill(q, k, v, tables, lens, qs, 0.3)
+    for b, L in enumerate(lens):
+        Q = q[qs[b]:qs[b + 1]].to(torch.float64).permute(1, 0, 2)        # [H, L, D]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            Q[None], _slab(k, b, MB, L)[None], _slab(v, b, MB, L)[None], scale=0.3,
+            is_causal=True, enable_gqa=True)[0].permute(1, 0, 2)
+        np.testing.assert_allclose(out[qs[b]:qs[b + 1]], ref.numpy(), rtol=RTOL, atol=1e-14)
+
+
+def test_prefill_chunk_is_the_tail_of_the_whole_prompt():
+    """Queries for the last n tokens give exactly the last n rows of the
+    whole-prompt prefill with the same query vectors (chunked prefill)."""
+    lens = (37, 22)
+    q, k, v, tables, lens, MB, qs = _prefill_case(50, lens, lens)
+    whole = oracle.paged_prefill(q, k, v, tables, lens, qs, 0.3)
+    for n in (1, 5, 16):
+        rows = np.concatenate([np.arange(qs[b + 1] - n, qs[b + 1]) for b in range(2)])
+        qs_n = np.array([0, n, 2 * n], dtype=np.int32)
+        part = oracle.paged_prefill(q[rows], k, v, tables, lens, qs_n, 0.3)
+        assert np.array_equal(part, whole[rows])
+
+
+def test_prefill_single_query_is_decode():
+    lens = (37, 9)
+    q, k, v, tables, lens, MB, qs = _prefill_case(51, lens, (1, 1))
+    pre = oracle.paged_prefill(q, k, v, tables, lens, qs, 0.3)
+    dec = oracle.paged_decode(q, k, v, tables, lens, 0.3)
+    assert np.array_equal(pre, dec)
+
+
+def test_prefill_closed_forms():
+    """Position 0 sees only token 0 (out = V_0 exactly); a zero query weighs the
+    causal prefix uniformly (out at position p = mean of V_0 .. V_p)."""
+    lens = (23, 14)
+    q, k, v, tables, lens, MB, qs = _prefill_case(52, lens, lens)
+    out = oracle.paged_prefill(q, k, v, tables, lens, qs, 0.7)
+    zero = oracle.paged_prefill(torch.zeros_like(q), k, v, tables, lens, qs, 0.7)
+    for b, L in enumerate(lens):
+        V = _slab(v, b, MB, L).numpy()                                  # [Hkv, L, D]
+        for h in range(4):
+            assert np.array_equal(out[qs[b], h], V[h // 2, 0])
+            prefix_mean = np.cumsum(V[h // 2], axis=0) / np.arange(1, L + 1)[:, None]
+            np.testing.assert_allclose(zero[qs[b]:qs[b + 1], h], prefix_mean, rtol=RTOL,
+                                       atol=1e-14)
+
+
+def test_prefill_block_permutation_invariance_is_bit_exact():
+    lens = (29, 17)
+    q, k, v, tables, lens, MB, qs = _prefill_case(53, lens, (11, 17))
+    base = oracle.paged_prefill(q, k, v, tables, lens, qs, 0.35)
+    perm = np.random.default_rng(3).permutation(k.shape[0])
+    k2, v2 = torch.empty_like(k), torch.empty_like(v)
+    k2[perm] = k
+    v2[perm] = v
+    moved = oracle.paged_prefill(q, k2, v2, perm[tables].astype(np.int32), lens, qs, 0.35)
+    assert np.array_equal(base, moved)
+
+
+def test_prefill_rejects_more_queries_than_context():
+    q, k, v, tables, lens, MB, qs = _prefill_case(54, (5, 3), (5, 4))
+    with pytest.raises(ValueError):
+        oracle.paged_prefill(q, k, v, tables, lens, qs, 0.3)
