@@ -64,6 +64,8 @@ typedef enum pkv_dtype { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
 #define PKV_DEVERR_BAD_SLOT 4        /* slot >= num_blocks*block_size: token skipped */
 #define PKV_DEVERR_WAIT_TIMEOUT 8    /* a pipeline wait ran past its iteration limit: work skipped */
 #define PKV_DEVERR_BAD_PAIR 16       /* copy pair id outside the pool: pair skipped */
+#define PKV_DEVERR_BAD_QUERY_COUNT 32 /* prefill: query count < 0 or > context length, or a query
+                                         row past num_tokens: clamped / not written */
 
 /* Shape of one KV pool (shared by the K and V pools). */
 typedef struct pkv_cache_desc {
@@ -185,6 +187,44 @@ pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* out, const v
                                   int32_t num_heads, float scale, int32_t partition_size,
                                   void* workspace, size_t workspace_bytes, int32_t* err_flag,
                                   void* stream);
+
+/*
+ * Paged prefill attention: the prompt phase through the same block table
+ * ([ops page] How it works: attention reads keys and values through the block
+ * table; Concept: processing the prompt is the compute-bound phase, generation
+ * the memory-bound one).  Sequence b holds context_lens[b] tokens in the pool,
+ * of which the last n_b = query_start[b + 1] - query_start[b] are this call's
+ * query tokens, their keys and values already appended (paged_kv_append).
+ * Query token i of sequence b sits at position p = context_lens[b] - n_b + i
+ * and attends causally to tokens 0 .. p:
+ *   out[query_start[b] + i][h][:] = sum_{t <= p} softmax_t(scale q . K[b][t]) V[b][t]
+ * with kv head h / (num_heads / num_kv_heads).  n_b = context_lens[b] is a
+ * whole prompt, n_b < context_lens[b] a chunk of one (chunked prefill), n_b = 1
+ * a single decode token, n_b = 0 nothing.
+ * Arithmetic: fp16/bf16 inputs; Q K^T and P V on the tensor cores with fp32
+ * accumulation; softmax in fp32 (base 2, scale * log2 e folded in); the
+ * probabilities enter P V rounded to `dtype`, except in the first 128-token
+ * tile of every sequence, where their rounding residual is added by a second
+ * product; output rounded to `dtype`.
+ *   out, q          device [num_tokens][num_heads][head_dim], 16-byte aligned;
+ *                   rows of a sequence are consecutive, sequences in order.
+ *   k_cache, v_cache device pools, 16-byte aligned (read only).
+ *   block_tables    device int32 [num_seqs][max_blocks_per_seq]; entries at or
+ *                   past ceil(context_len / block_size) are not read.
+ *   context_lens    device int32 [num_seqs].
+ *   query_start     device int32 [num_seqs + 1], query_start[num_seqs] = num_tokens.
+ *   num_heads / num_kv_heads must be a power of two <= 128.
+ *   err_flag        device int32 or NULL (PKV_DEVERR_BAD_BLOCK_ID,
+ *                   PKV_DEVERR_BAD_CONTEXT_LEN, PKV_DEVERR_BAD_QUERY_COUNT,
+ *                   PKV_DEVERR_WAIT_TIMEOUT).
+ * Needs no workspace.  num_tokens == 0 enqueues nothing.
+ */
+pkv_status paged_attention_prefill(const pkv_cache_desc* desc, void* out, const void* q,
+                                   const void* k_cache, const void* v_cache,
+                                   const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                   const int32_t* context_lens, const int32_t* query_start,
+                                   int32_t num_seqs, int32_t num_tokens, int32_t num_heads,
+                                   float scale, int32_t* err_flag, void* stream);
 
 /*
  * Decode without a caller workspace, for callers that cannot allocate device

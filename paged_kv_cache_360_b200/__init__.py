@@ -21,7 +21,7 @@ from ._lib import PkvError, PoolExhausted  # noqa: F401
 __all__ = [
     "paged_kv_append", "copy_blocks", "swap_blocks", "paged_attention_decode",
     "paged_attention_workspace_bytes",
-    "paged_attention_decode_static_scratch", "Pool",
+    "paged_attention_decode_static_scratch", "paged_attention_prefill", "Pool",
     "PkvError", "PoolExhausted", "launch_count", "cache_desc",
 ]
 
@@ -168,6 +168,28 @@ def paged_attention_decode_static_scratch(out, q, k_cache, v_cache, block_tables
         int(block_tables.shape[1]), _dev(context_lens, "context_lens", torch.int32), B, H,
         ctypes.c_float(scale), int(partition_size), _dev(err_flag, "err_flag", torch.int32),
         _stream(stream)))
+    return out
+
+
+def paged_attention_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
+                            scale, err_flag=None, stream=None):
+    """Causal prefill through the block tables: q and out are [T, H, D] with
+    sequence b's query tokens in rows query_start[b] .. query_start[b+1]-1, the
+    last ones of its context_lens[b] tokens (already appended).  Returns `out`."""
+    torch = _torch()
+    desc = cache_desc(k_cache)
+    T, H, D = q.shape
+    if tuple(out.shape) != (T, H, D) or out.dtype != q.dtype or q.dtype != k_cache.dtype:
+        raise PkvError(1, "q and out must be [T, H, D] of the cache dtype")
+    B = int(context_lens.shape[0])
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or query_start.shape[0] != B + 1:
+        raise PkvError(1, "block_tables must be [B, MB], context_lens [B], query_start [B + 1]")
+    _lib.check(_lib.load().paged_attention_prefill(
+        ctypes.byref(desc), _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"),
+        _dev(v_cache, "v_cache"), _dev(block_tables, "block_tables", torch.int32),
+        int(block_tables.shape[1]), _dev(context_lens, "context_lens", torch.int32),
+        _dev(query_start, "query_start", torch.int32), B, T, H, ctypes.c_float(scale),
+        _dev(err_flag, "err_flag", torch.int32), _stream(stream)))
     return out
 
 

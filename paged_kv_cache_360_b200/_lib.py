@@ -25,7 +25,7 @@ STATIC_SCRATCH_BYTES = 16 << 20
 # Every function include/pkv.h declares (checked by the tests against the header).
 EXPORTS = (
     "paged_kv_append", "copy_blocks", "swap_blocks", "paged_attention_workspace_bytes", "paged_attention_decode",
-    "paged_attention_decode_static_scratch",
+    "paged_attention_decode_static_scratch", "paged_attention_prefill",
     "pkv_pool_create", "pkv_pool_destroy", "pkv_seq_new", "pkv_seq_fork", "pkv_seq_reserve",
     "pkv_seq_reserve_tokens", "pkv_seq_new_cached",
     "pkv_seq_cow", "pkv_seq_free", "pkv_seq_swap_out", "pkv_seq_swap_in", "pkv_seq_len", "pkv_seq_block_table", "pkv_pool_block_tables",
@@ -83,6 +83,8 @@ def load():
                                                 ctypes.c_float, i32, p, sz, p, p]),
                 "paged_attention_decode_static_scratch": (st, [P(CacheDesc), p, p, p, p, p, i32, p,
                                                                i32, i32, ctypes.c_float, i32, p, p]),
+                "paged_attention_prefill": (st, [P(CacheDesc), p, p, p, p, p, i32, p, p, i32, i32,
+                                                 i32, ctypes.c_float, p, p]),
                 "pkv_pool_create": (st, [i32, i32, p, P(p)]),
                 "pkv_pool_destroy": (None, [p]),
                 "pkv_seq_new": (st, [p, P(i32)]),
