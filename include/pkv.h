@@ -98,8 +98,9 @@ pkv_status paged_kv_append(const pkv_cache_desc* desc, void* k_cache, void* v_ca
 /*
  * Copy-on-write block copy: for each pair (src, dst) copy block src over block
  * dst -- every kv head and offset -- in both pools ([ops page] How it works:
- * sequences that share blocks "only copy-on-write when they diverge"; At a
- * glance: a block is copied only when a sequence writes to it).
+ * sequences that share blocks get private copies only once their contents
+ * differ; At a glance: a shared block is duplicated when one of its sequences
+ * writes into it).
  *   block_mapping  device int32 [num_pairs][2] = (src, dst).  Destinations must
  *                  be distinct and no destination may be a source (pairs run
  *                  concurrently); the host block manager's pairs always are.
@@ -150,9 +151,9 @@ size_t paged_attention_workspace_bytes(const pkv_cache_desc* desc, int32_t num_s
 /*
  * Paged decode attention: one query token per sequence attends over its
  * context, reading keys and values through the block table ([ops page] How it
- * works: the kernel "reads KV through the block table, gathering scattered
- * physical blocks"; Concept: the block table maps logical positions to
- * physical blocks; [glossary]).
+ * works: the attention kernel fetches keys and values block by block through
+ * the table, wherever the blocks lie; Concept: the block table maps logical
+ * positions to physical blocks; [glossary]).
  *   out[b][h][:] = sum_t softmax_t(scale * q[b][h] . K[b][t]) V[b][t],
  *   t < context_lens[b], K/V of logical token t read from physical block
  *   block_tables[b][t / block_size] at offset t % block_size, kv head

@@ -15,9 +15,10 @@
  * What is computed here is the plain definition, written out with no
  * blocking, fusion or reordering:
  *   - gather: a sequence's logical token t lives in physical block
- *     table[t / bs] at offset t % bs ([ops page] Concept: "a per-sequence block
- *     table maps logical positions to physical blocks"; How it works: the kernel
- *     "reads KV through the block table, gathering scattered physical blocks");
+ *     table[t / bs] at offset t % bs ([ops page] Concept: every sequence has a
+ *     table from its logical positions to physical blocks; How it works: the
+ *     attention kernel fetches keys and values block by block through that
+ *     table, wherever the blocks lie);
  *   - attention of one query over the gathered keys and values, softmax with
  *     the maximum subtracted, in double precision;
  *   - the append and block-copy steps as byte copies ([ops page] How it works:
@@ -29,7 +30,7 @@
  *     separate pools;
  *   - query head h reads kv head h / (num_heads / num_kv_heads);
  *   - context_len counts the token appended in the same step; 0 gives zeros;
- *   - a negative slot in the append mapping means "skip this token";
+ *   - a negative slot in the append mapping means the token is skipped;
  *   - fp16 / bf16 storage values are widened exactly to double.
  *
  * Parity status: every exported function is pinned by tests under tests/
@@ -326,8 +327,9 @@ int oracle_paged_prefill(int dtype, const uint16_t* q, const uint16_t* k_cache,
 /*
  * Append: write token i's key and value rows (every kv head) into slot
  * slot_mapping[i] of the pool, i.e. physical block slot / bs at offset
- * slot % bs ([ops page] How it works: "writes the new token's key and value
- * into the sequence's current block").  A negative slot skips the token.
+ * slot % bs ([ops page] How it works: each step stores the new token's key and
+ * value in the block the sequence is currently filling).  A negative slot skips
+ * the token.
  *   key, value: [N][Hkv][D] storage words; caches as above, modified in place.
  * Returns 0, or -1 if a slot is past the pool.
  */
