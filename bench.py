@@ -39,6 +39,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention KV GB/s (% of B200 HBM peak); seq-decode-steps/sec"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -432,6 +433,245 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
+# ------------------------------------------------------------------ prefill
+
+PREFILL_METRIC = "paged prefill attention TFLOP/s (causal, % of B200 bf16 dense peak)"
+
+
+def build_prefill_step(wl, pkv):
+    """Block tables, lengths and the query tokens' slots from the library's
+    block manager: every sequence first holds its earlier context, then
+    reserves its query tokens."""
+    pool = pkv.Pool(wl.num_blocks, wl.block_size, wl.free_order)
+    seqs = []
+    nq = np.diff(wl.query_start)
+    for b in range(wl.num_seqs):
+        s = pool.new_seq()
+        pool.reserve(s, int(wl.context_lens[b] - nq[b]))
+        seqs.append(s)
+    slots = []
+    for b, s in enumerate(seqs):
+        sl, cp = pool.reserve(s, int(nq[b]))
+        assert not cp
+        slots.extend(int(x) for x in sl)
+    mb = max(len(pool.table(s)) for s in seqs)
+    tables, lens = pool.block_tables(seqs, mb, pad=-1)
+    pool.close()
+    return np.asarray(slots, dtype=np.int64), tables, lens
+
+
+def prefill_flops(lens, query_start, H, D) -> int:
+    """Causal attention FLOPs: 2 D for q . k and 2 D for p v per (query row,
+    visible key) pair and head."""
+    nq = np.diff(np.asarray(query_start, dtype=np.int64))
+    L = np.asarray(lens, dtype=np.int64)
+    pairs = nq * (L - nq) + nq * (nq + 1) // 2
+    return int(pairs.sum()) * 4 * H * D
+
+
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0.0)), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def run_prefill(args, rank, world, local_rank):
+    import paged_kv_cache_360_b200 as pkv
+    from paged_kv_cache_360_b200.workloads import make_prefill_workload
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = make_prefill_workload(args.prefill_workload, seed=args.seed, rank=rank)
+    slots, tables, lens = build_prefill_step(wl, pkv)
+    k, v = wl.k_cache.to(dev), wl.v_cache.to(dev)
+    q, key, value = wl.q.to(dev), wl.new_key.to(dev), wl.new_value.to(dev)
+    d_slots = torch.from_numpy(slots).to(dev)
+    d_tables = torch.from_numpy(tables).to(dev)
+    d_lens = torch.from_numpy(lens).to(dev)
+    d_qs = torch.from_numpy(wl.query_start).to(dev)
+    out = torch.empty_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def append():
+        pkv.paged_kv_append(k, v, key, value, d_slots, err_flag=err)
+
+    def attend():
+        pkv.paged_attention_prefill(out, q, k, v, d_tables, d_lens, d_qs, wl.scale, err_flag=err)
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        n0 = pkv.launch_count()
+        append()
+        attend()
+        launches_per_step = pkv.launch_count() - n0
+    torch.cuda.synchronize()
+    g_step, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=stream):
+        append()
+        attend()
+    with torch.cuda.graph(g_attn, stream=stream):
+        attend()
+    torch.cuda.synchronize()
+    flops = prefill_flops(lens, wl.query_start, wl.num_heads, wl.head_dim)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def timed(graph, steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(steps):
+                graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return e0.elapsed_time(e1)
+
+    sampler = ClockSampler()
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            g_step.replay()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    step_ms = timed(g_step, args.steps)
+    t_wall1 = time.time()
+    attn_ms = timed(g_attn, args.steps)
+
+    # end to end: pinned host inputs -> device, append + prefill, output -> pinned host
+    h_in = [t.pin_memory() for t in (wl.q, wl.new_key, wl.new_value, torch.from_numpy(slots),
+                                     torch.from_numpy(tables), torch.from_numpy(lens),
+                                     torch.from_numpy(wl.query_start))]
+    d_in = [torch.empty_like(t, device=dev) for t in h_in]
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2e_out = torch.empty_like(out)
+
+    def e2e_step():
+        for h, d in zip(h_in, d_in):
+            d.copy_(h, non_blocking=True)
+        pkv.paged_kv_append(k, v, d_in[1], d_in[2], d_in[3], err_flag=err)
+        pkv.paged_attention_prefill(e2e_out, d_in[0], k, v, d_in[4], d_in[5], d_in[6], wl.scale,
+                                    err_flag=err)
+        h_out.copy_(e2e_out, non_blocking=True)
+
+    g_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_e2e, stream=stream):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(3, min(args.steps, 500))
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            g_e2e.replay()
+    e2e_ms = timed(g_e2e, e2e_steps)
+    if rank == 0:
+        sampler.stop()
+    torch.cuda.synchronize()
+    err_val = int(err.item())
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = h_out.numel() * h_out.element_size()
+
+    step_ms, attn_ms, e2e_ms = max_over_ranks([step_ms, attn_ms, e2e_ms], world, dev)
+    if rank != 0:
+        return None
+    peak, peak_sustained, peak_kind = measured_tensor_peak()
+    ms_per_step = step_ms / args.steps
+    attn_avg = attn_ms / args.steps
+    achieved = flops / (attn_avg * 1e-3) / 1e12
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    e2e_per_step = e2e_ms / e2e_steps
+    nq = np.diff(wl.query_start)
+    line = {
+        "metric": PREFILL_METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "num_seqs_per_gpu": wl.num_seqs,
+                   "query_tokens_per_gpu": wl.num_tokens, "num_heads": wl.num_heads,
+                   "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+                   "block_size": wl.block_size, "num_blocks": wl.num_blocks,
+                   "context_lens": [int(x) for x in lens],
+                   "query_counts": [int(x) for x in nq], "seed": args.seed,
+                   "parallelism": f"dp{world} (independent batches per GPU)",
+                   "l2": "not flushed: the pool is %.0f MB, %.1fx the 126 MB L2"
+                         % (2 * k.numel() * k.element_size() / 1e6,
+                            2 * k.numel() * k.element_size() / 126e6),
+                   "timing": "CUDA events around K back-to-back replays of the step's CUDA graph "
+                             "(paged_kv_append of the query tokens' K/V, then the prefill)"},
+        "attention_flops_per_step": flops,
+        "roofline": {"bound": "tensor", "kernel": "paged_attention_prefill (tcgen05)",
+                     "timing": "CUDA events around K back-to-back prefill-only graph replays",
+                     "achieved": round(achieved, 2), "peak": peak,
+                     "peak_kind": f"{peak_kind} bf16 dense burst",
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "frac_of_sustained": round(achieved / peak_sustained, 4) if peak_sustained else None,
+                     "traffic": None, "algorithmic_flops_per_launch": flops,
+                     "avg_launch_ms": round(attn_avg, 5)},
+        "e2e": {"value": round(world * flops / (e2e_per_step * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_per_step, 5), "steps": e2e_steps,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "path": "per step: pinned host -> device copies of q, the new K/V, slots, tables, "
+                        "lengths and query starts; paged_kv_append; paged_attention_prefill; "
+                        "device -> pinned host copy of the output; one stream, one CUDA graph"},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "launches_per_step": int(launches_per_step),
+        "device_err_flag": err_val,
+        "clocks": sampler.summary(t_wall0, t_wall1),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = prefill_cpu_baseline(wl, slots, tables, lens, args.cpu_budget)
+    return line
+
+
+def prefill_cpu_baseline(wl, slots, tables, lens, budget_s):
+    """The oracle's append + prefill on a bounded sample: the last m query
+    tokens of the first chunked request (the prefill of a chunk of m tokens),
+    m grown until about `budget_s` of CPU time."""
+    import oracle
+    oracle.build()
+    nq = np.diff(wl.query_start)
+    b = 1 if wl.num_seqs > 1 else 0
+    L = int(lens[b])
+    kw, vw = oracle.words(wl.k_cache), oracle.words(wl.v_cache)
+    r0, r1 = int(wl.query_start[b]), int(wl.query_start[b + 1])
+    oracle.append(kw, vw, wl.new_key[r0:r1], wl.new_value[r0:r1], slots[r0:r1])
+
+    def sample(m):
+        qs = np.array([0, m], dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.paged_prefill(wl.q[r1 - m:r1], kw, vw, tables[b:b + 1], lens[b:b + 1], qs, wl.scale)
+        return time.perf_counter() - t0
+
+    m = 1
+    dt = sample(m)
+    while m < int(nq[b]) and dt * 2 < budget_s:
+        m = min(int(nq[b]), m * 2)
+        dt = sample(m)
+    fl = prefill_flops([L], [0, m], wl.num_heads, wl.head_dim)
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "seconds": round(dt, 3),
+            "sample": f"oracle prefill of the last {m} query tokens of request {b} "
+                      f"(context {L}) of the {wl.name} batch, single-threaded C float64"}
+
+
 # ------------------------------------------------------ CPU oracle (baseline)
 
 def sample_bytes(wl, sub_lens, n) -> int:
@@ -543,6 +783,9 @@ def main():
                     help="0 = balanced split (default unless the workload fixes one); "
                          "> 0 = fixed partitions of that many tokens")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["decode", "prefill"], default="decode",
+                    help="decode: the decode step (default); prefill: the paged prefill step")
+    ap.add_argument("--prefill-workload", default="prefill-llama3-8b-layer")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU time")
     ap.add_argument("--ref-step-budget", type=float, default=3.0,
@@ -568,7 +811,8 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, rank, world, local_rank)
+        run = run_prefill if args.workload == "prefill" else run_ours
+        line = run(args, rank, world, local_rank)
         if line is not None:
             print(json.dumps(line), flush=True)
     finally:

@@ -280,3 +280,78 @@ def random_block_pairs(rng: np.random.Generator, num_blocks: int, m: int) -> np.
 def shard_seed(seed: int, rank: int) -> tuple[int, int]:
     """Each rank of a multi-GPU run draws its own batch: (seed, rank) keys the draw."""
     return int(seed), int(rank)
+
+
+# ------------------------------------------------------------------ prefill
+
+PREFILL_CONFIGS = {
+    # 16 requests of a Llama-3-8B layer: half are whole prompts, half a 512-token
+    # chunk at the end of a longer context (chunked prefill)
+    "prefill-llama3-8b-layer": dict(B=16, H=32, Hkv=8, D=128, bs=16, dtype=BF16, lo=512,
+                                    hi=4096, chunk=512),
+    # small case for the oracle
+    "prefill-tiny": dict(B=4, H=8, Hkv=2, D=128, bs=16, dtype=BF16, lo=1, hi=300, chunk=64),
+}
+
+
+@dataclass
+class PrefillWorkload:
+    """One batch of prefill inputs on the host.
+
+    Sequence b holds ``context_lens[b]`` tokens; its last ``n_b =
+    query_start[b+1] - query_start[b]`` are the step's query tokens, whose keys
+    and values are rows ``query_start[b] ..`` of ``new_key`` / ``new_value``.
+    The earlier tokens' keys and values are whatever the pool holds.  Block ids
+    are handed out by a block manager seeded with ``free_order``."""
+
+    name: str
+    seed: int
+    rank: int
+    num_seqs: int
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    dtype: torch.dtype
+    scale: float
+    context_lens: np.ndarray
+    query_start: np.ndarray
+    free_order: np.ndarray
+    q: torch.Tensor | None = None
+    k_cache: torch.Tensor | None = None
+    v_cache: torch.Tensor | None = None
+    new_key: torch.Tensor | None = None
+    new_value: torch.Tensor | None = None
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.query_start[-1])
+
+
+def make_prefill_workload(name: str = "prefill-llama3-8b-layer", seed: int = 0, rank: int = 0,
+                          materialize: bool = True) -> PrefillWorkload:
+    """Lengths L ~ U[lo, hi]; even-indexed requests query their whole prompt,
+    odd-indexed ones the last min(chunk, L) tokens.  The pool has 3 % more
+    blocks than the contexts fill, ids in a seeded random order."""
+    c = PREFILL_CONFIGS[name]
+    rng = np.random.default_rng([int(seed), 1000 + list(PREFILL_CONFIGS).index(name), int(rank)])
+    B, bs = c["B"], c["bs"]
+    lens = rng.integers(c["lo"], c["hi"] + 1, size=B).astype(np.int32)
+    nq = np.where(np.arange(B) % 2 == 0, lens, np.minimum(lens, c["chunk"])).astype(np.int32)
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    used = int(sum(_blocks_for(x, bs) for x in lens))
+    num_blocks = int(math.ceil(used * 1.03)) + 1
+    wl = PrefillWorkload(
+        name=name, seed=seed, rank=rank, num_seqs=B, num_heads=c["H"], num_kv_heads=c["Hkv"],
+        head_dim=c["D"], block_size=bs, num_blocks=num_blocks, dtype=c["dtype"],
+        scale=float(np.float32(1.0 / math.sqrt(c["D"]))), context_lens=lens, query_start=qs,
+        free_order=rng.permutation(num_blocks).astype(np.int32))
+    if materialize:
+        T = int(qs[-1])
+        wl.q = normal_tensor(rng, (T, c["H"], c["D"]), c["dtype"])
+        wl.k_cache = normal_tensor(rng, (num_blocks, c["Hkv"], bs, c["D"]), c["dtype"])
+        wl.v_cache = normal_tensor(rng, (num_blocks, c["Hkv"], bs, c["D"]), c["dtype"])
+        wl.new_key = normal_tensor(rng, (T, c["Hkv"], c["D"]), c["dtype"])
+        wl.new_value = normal_tensor(rng, (T, c["Hkv"], c["D"]), c["dtype"])
+    return wl
