@@ -186,11 +186,23 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def decode_device_sha256() -> str:
+    """Hash of the decode kernels' device code: pkv_decode.cu up to its host
+    section, and the device headers it includes."""
+    import hashlib
+    csrc = os.path.join(ROOT, "paged_kv_cache_360_b200", "csrc")
+    h = hashlib.sha256()
+    src = open(os.path.join(csrc, "pkv_decode.cu"), "rb").read()
+    h.update(src[:src.find(b"// ------------------------------------------------------------------ host side")])
+    for name in ("pkv_attend.cuh", "pkv_ptx.cuh"):
+        h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()
+
+
 def traffic_record():
     """DRAM bytes per decode launch from the committed ncu summary
     profiles/decode_traffic.txt, if it was taken on the current decode source
     (else None)."""
-    import hashlib
     path = os.path.join(ROOT, "profiles", "decode_traffic.txt")
     try:
         rec = {}
@@ -200,8 +212,7 @@ def traffic_record():
                 rec[key.strip()] = val.strip()
     except OSError:
         return None
-    src = open(os.path.join(ROOT, "paged_kv_cache_360_b200", "csrc", "pkv_decode.cu"), "rb").read()
-    if rec.get("source_sha256") != hashlib.sha256(src).hexdigest():
+    if rec.get("source_sha256") != decode_device_sha256():
         return None
     return {"bytes_per_launch": int(rec["bytes_per_launch"])}
 
