@@ -105,3 +105,28 @@ def test_append_and_copy_reject_bad_arguments(lib):
 def test_status_strings(lib):
     for code, name in _lib.STATUS_NAMES.items():
         assert lib.pkv_status_string(code).decode() == name
+
+
+def _prefill(lib, desc, **kw):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, tables=FAKE, mb=4, lens=FAKE, qs=FAKE, B=2, T=40,
+             H=4, scale=0.1)
+    a.update(kw)
+    return lib.paged_attention_prefill(ctypes.byref(desc), a["out"], a["q"], a["k"], a["v"],
+                                       a["tables"], a["mb"], a["lens"], a["qs"], a["B"], a["T"],
+                                       a["H"], ctypes.c_float(a["scale"]), None, None)
+
+
+def test_prefill_rejects_bad_arguments(lib):
+    d = _desc()
+    assert _prefill(lib, _desc(head_dim=96)) == 2
+    assert _prefill(lib, d, H=3) == 1                    # not a multiple of num_kv_heads
+    assert _prefill(lib, d, H=6) == 2                    # group 3: not a power of two
+    assert _prefill(lib, d, H=2 * 256) == 2              # group 256 > 128
+    assert _prefill(lib, d, scale=float("inf")) == 1
+    assert _prefill(lib, d, T=-1) == 1
+    assert _prefill(lib, d, mb=0) == 1
+    assert _prefill(lib, d, qs=None) == 1
+    assert _prefill(lib, d, out=ctypes.c_void_p(0x10008)) == 1   # misaligned
+    assert _prefill(lib, d, T=0) == 0                    # nothing to do
+    assert _prefill(lib, d, B=0) == 0
+    assert lib.pkv_last_error().decode()
