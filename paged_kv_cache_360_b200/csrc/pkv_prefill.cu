@@ -258,41 +258,58 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
         if (warp == 0) {
             // ------------------------------------------------------ producer
+            // Table entries come 32 at a time (one per lane, one coalesced
+            // load), the next 32 prefetched while the current ones are used;
+            // lane l issues the copies of block l of each kv tile.
+            constexpr int kBlocksPerTile = kPfKv / BS;
+            constexpr int kTilesPerChunk = 32 / kBlocksPerTile;
+            const int32_t* row = a.tables + static_cast<int64_t>(b) * a.max_blocks;
+            auto load_chunk = [&](int c) {
+                const int idx = c * 32 + lane;
+                int id = 0;  // blocks past the context: any valid block, masked
+                if (idx * BS < L) {
+                    id = __ldg(row + idx);
+                    if (id < 0 || id >= a.num_blocks) {
+                        flag(a.err, PKV_DEVERR_BAD_BLOCK_ID);
+                        id = 0;
+                    }
+                }
+                return id;
+            };
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar(kBarQ), Lay::kTile);
                 tma_load_4d(sb + Lay::kQ, &tq, 0, hk * g, q0 + t_lo, 0, bar(kBarQ));
-                const int32_t* row = a.tables + static_cast<int64_t>(b) * a.max_blocks;
-                int issued = 0;
-                for (int j = 0; j < nkv; ++j) {
-                    const int s = j % kPfStages;
-                    if (j >= kPfStages &&
-                        !one_wait(bar(kBarKvEmpty + s), ((j / kPfStages) - 1) & 1, abort_word, a.err))
-                        break;
-                    const uint32_t ks = sb + Lay::kStage0 + 2u * s * Lay::kTile;
-                    const uint32_t vs = ks + Lay::kTile;
-                    mbar_arrive_expect_tx(bar(kBarKvFull + s), 2u * Lay::kTile);
-#pragma unroll 1
-                    for (int blk = 0; blk < kPfKv / BS; ++blk) {
-                        const int tok = j * kPfKv + blk * BS;
-                        int id = 0;  // blocks past the context: any valid block, masked
-                        if (tok < L) {
-                            id = __ldg(row + tok / BS);
-                            if (id < 0 || id >= a.num_blocks) {
-                                flag(a.err, PKV_DEVERR_BAD_BLOCK_ID);
-                                id = 0;
-                            }
-                        }
-                        const int y = (id * a.num_kv_heads + hk) * BS;
-#pragma unroll
-                        for (int h = 0; h < Lay::kHalves; ++h) {
-                            const uint32_t off = h * Lay::kHalfBytes + blk * BS * 128;
-                            tma_load_3d(ks + off, &tk, 0, y, h, bar(kBarKvFull + s));
-                            tma_load_3d(vs + off, &tv, 0, y, h, bar(kBarKvFull + s));
-                        }
-                    }
-                    issued = j + 1;
+            }
+            int cur = load_chunk(0), next = 0;
+            int issued = 0;
+            for (int j = 0; j < nkv; ++j) {
+                const int s = j % kPfStages;
+                if (j % kTilesPerChunk == 0) {
+                    if (j > 0) cur = next;
+                    next = load_chunk(j / kTilesPerChunk + 1);
                 }
-                // Let every copy in flight land before the CTA can exit.
+                if (j >= kPfStages &&
+                    !warp_wait(bar(kBarKvEmpty + s), ((j / kPfStages) - 1) & 1, abort_word, a.err))
+                    break;
+                const uint32_t ks = sb + Lay::kStage0 + 2u * s * Lay::kTile;
+                const uint32_t vs = ks + Lay::kTile;
+                if (lane == 0) mbar_arrive_expect_tx(bar(kBarKvFull + s), 2u * Lay::kTile);
+                __syncwarp();
+                const int id = __shfl_sync(0xffffffffu, cur,
+                                           (j % kTilesPerChunk) * kBlocksPerTile + (lane % kBlocksPerTile));
+                if (lane < kBlocksPerTile) {
+                    const int y = (id * a.num_kv_heads + hk) * BS;
+#pragma unroll
+                    for (int h = 0; h < Lay::kHalves; ++h) {
+                        const uint32_t off = h * Lay::kHalfBytes + lane * BS * 128;
+                        tma_load_3d(ks + off, &tk, 0, y, h, bar(kBarKvFull + s));
+                        tma_load_3d(vs + off, &tv, 0, y, h, bar(kBarKvFull + s));
+                    }
+                }
+                issued = j + 1;
+            }
+            // Let every copy in flight land before the CTA can exit.
+            if (lane == 0) {
                 for (uint32_t i = 0; i < kWaitLimit && !mbar_test(bar(kBarQ), 0); ++i) {
                 }
                 for (int j = issued - kPfStages < 0 ? 0 : issued - kPfStages; j < issued; ++j)
@@ -395,13 +412,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 // S buffer (j & 1) is free once every lane has read it; the
                 // arrival on P-full below publishes that to the MMA issuer.
                 const int kv0 = j * kPfKv;
-                float mt = -INFINITY;
+                float mx[8];
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    const float v = kv0 + c <= p ? __uint_as_float(x[c]) * sl2 : -INFINITY;
-                    x[c] = __float_as_uint(v);
-                    mt = fmaxf(mt, v);
+                for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+                if (kv0 + kPfKv - 1 <= p) {  // the whole tile is visible to this row
+#pragma unroll
+                    for (int c = 0; c < 128; ++c) {
+                        const float v = __uint_as_float(x[c]) * sl2;
+                        x[c] = __float_as_uint(v);
+                        mx[c & 7] = fmaxf(mx[c & 7], v);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c) {
+                        const float v = kv0 + c <= p ? __uint_as_float(x[c]) * sl2 : -INFINITY;
+                        x[c] = __float_as_uint(v);
+                        mx[c & 7] = fmaxf(mx[c & 7], v);
+                    }
                 }
+                const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
                 const bool rescale = mt > m_used + kRescaleLog2;
                 float factor = 1.f;
                 if (rescale) {
@@ -410,18 +440,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     l *= factor;
                 }
                 uint32_t hi[64], lo[64];
-                float sum = 0.f;
+                float sm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int i = 0; i < 64; ++i) {
                     const float p0 = exp2_approx(__uint_as_float(x[2 * i]) - m_used);
                     const float p1 = exp2_approx(__uint_as_float(x[2 * i + 1]) - m_used);
-                    sum += p0;
-                    sum += p1;
+                    sm[i & 3] += p0 + p1;
                     float r0, r1, q0_, q1_;
                     hi[i] = Pack<T>::two(p0, p1, r0, r1);
                     lo[i] = j == 0 ? Pack<T>::two(p0 - r0, p1 - r1, q0_, q1_) : 0u;
                 }
-                l += sum;
+                l += (sm[0] + sm[1]) + (sm[2] + sm[3]);
                 // The previous P V must be done: it reads the P tile and writes O.
                 if (ev > 0 && !(ok = warp_wait(bar(kBarODone), (ev - 1) & 1, abort_word, a.err)))
                     break;
