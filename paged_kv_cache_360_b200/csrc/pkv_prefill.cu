@@ -5,23 +5,29 @@
 // prompt processing is the compute-bound phase): the last n_b tokens of every
 // sequence attend causally to the sequence's paged context.
 //
-// One CTA computes one tile of 128 query rows against all the kv tiles it can
-// see.  The rows are (token, head) pairs of one kv head: 128 / g consecutive
-// query tokens times the g query heads that share the kv head, so every key and
-// value row fetched serves g heads.  Per CTA:
-//   warp 0      producer: the Q tile once (one 4-D TMA box), then per 128-token
-//               kv tile one 3-D TMA box per (block, 64-column half) of K and V
-//               into a two-stage ring;
-//   warp 1      MMA issuer (one thread) and tensor-memory owner:
-//               S_j = Q K_j^T into one of two 128-column TMEM buffers, then
-//               O += P_j V_j into a D-column TMEM accumulator;
-//   warps 2-5   softmax, one S row per thread (TMEM lane = row): mask, running
-//               maximum (rescaling O in TMEM only when the maximum grows by more
-//               than 2^8), P_j = 2^(s - m) rounded into a 128x128 shared tile
-//               for the next MMA, and at the end O / l to global memory.
-// S_{j+1} is computed while the softmax of tile j runs.  In tile 0 the softmax
-// also sends the rounding residual of P as a second P V product, so that rows
-// with few tokens (the start of every prompt) are accurate to fp32 weights.
+// A query tile is 128 rows: 128 / g consecutive query tokens times the g query
+// heads that share one kv head, so every key and value row fetched serves g
+// heads.  One CTA takes two neighbouring query tiles of one (sequence, kv
+// head) -- tile 0 the later one, tile 1 the one before it -- against the same
+// stream of 128-token kv tiles, so each K/V tile is loaded once for 256 rows and
+// the tensor core alternates between the tiles while each tile's softmax runs:
+//   warp 0      producer: both Q tiles (4-D TMA boxes), then per kv tile one
+//               3-D TMA box per (block, 64-column half) of K and of V into two
+//               2-stage rings (K freed by Q K^T, V by P V), K one tile ahead;
+//   warp 1      MMA issuer (one thread) and tensor-memory owner.  Per tile t:
+//               S_t = Q_t K_j^T (fp32, 128 TMEM columns), then O_t += P_t V_j
+//               with P_t read from tensor memory, O_t in its own 128 columns;
+//               order: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ...
+//   warps 2-5   softmax of tile 0, warps 6-9 of tile 1; one row per thread
+//               (TMEM lane = row): causal mask, running maximum, P = 2^(s - m)
+//               rounded to the input type and written back over S's first 64
+//               columns; in a sequence's first kv tile the rounding residual
+//               goes to columns 64-127 and enters P V as a second product.  O is
+//               rescaled in tensor memory only when the maximum grows by more
+//               than 2^8.  The MMAs of one thread complete in issue order, so
+//               when S_t(j) is complete so is P_t V(j-1): O_t is stable during
+//               the softmax and needs no extra wait.  At the end, O / l goes to
+//               global memory.
 //
 // Every mbarrier wait is bounded and warp-uniform; a timeout raises a shared
 // abort word, records PKV_DEVERR_WAIT_TIMEOUT and every role drains its
@@ -44,22 +50,23 @@
 namespace pkv {
 namespace {
 
-constexpr int kPfThreads = 192;      // producer warp, MMA warp, 4 softmax warps
-constexpr int kPfRows = 128;         // MMA M: query rows per CTA
+constexpr int kPfThreads = 320;      // producer warp, MMA warp, 2 softmax warpgroups
+constexpr int kPfRows = 128;         // MMA M: query rows per tile
 constexpr int kPfKv = 128;           // kv tokens per tile: N of Q K^T, K of P V
-constexpr int kPfStages = 2;         // K/V ring depth
-constexpr uint32_t kTmemCols = 512;  // S buffers at columns 0 and 128, O at 256
-constexpr uint32_t kTmemO = 256;
+constexpr int kPfStages = 2;         // K and V ring depth
+constexpr uint32_t kTmemCols = 512;  // S_t at 128 t, O_t at 256 + 128 t
 constexpr float kRescaleLog2 = 8.f;  // rescale O when the maximum grows by > 2^8
 
 enum : int {
     kBarQ = 0,
-    kBarKvFull = 1,
-    kBarKvEmpty = kBarKvFull + kPfStages,
-    kBarSFull = kBarKvEmpty + kPfStages,  // two
-    kBarPFull = kBarSFull + 2,
-    kBarODone,
-    kBarDrain,
+    kBarKFull = 1,
+    kBarKEmpty = kBarKFull + kPfStages,
+    kBarVFull = kBarKEmpty + kPfStages,
+    kBarVEmpty = kBarVFull + kPfStages,
+    kBarSFull = kBarVEmpty + kPfStages,  // per query tile
+    kBarPFull = kBarSFull + 2,           // per query tile, 128 arrivals
+    kBarODone = kBarPFull + 2,           // per query tile
+    kBarDrain = kBarODone + 2,
     kNumBars
 };
 
@@ -70,10 +77,9 @@ struct PfLayout {
     static constexpr int kHalves = D / 64;
     static constexpr int kHalfBytes = 128 * 128;
     static constexpr int kTile = kHalves * kHalfBytes;          // 128 rows x D
-    static constexpr int kQ = 0;
-    static constexpr int kStage0 = kTile;                       // stage s: K, then V
-    static constexpr int kP = kStage0 + 2 * kPfStages * kTile;  // 128 x 128 probabilities
-    static constexpr int kBars = kP + 2 * kHalfBytes;
+    static constexpr int kQ = 0;                                // two Q tiles
+    static constexpr int kStage0 = 2 * kTile;                   // stage s: K, then V
+    static constexpr int kBars = kStage0 + 2 * kPfStages * kTile;
     static constexpr int kMisc = kBars + 8 * kNumBars;  // tmem base, abort word, work item
     static constexpr int kBytes = kMisc + 32;
     static constexpr int kAlloc = kBytes + 1024;        // room to align the base
@@ -119,7 +125,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
     return ok;
 }
 
-// Single-thread variant (producer, MMA issuer).
+// Single-thread variant (MMA issuer).
 __device__ __forceinline__ bool one_wait(uint32_t bar, uint32_t parity,
                                          volatile uint32_t* abort_word, int32_t* err) {
     for (uint32_t i = 0; i < kWaitLimit; ++i) {
@@ -131,6 +137,12 @@ __device__ __forceinline__ bool one_wait(uint32_t bar, uint32_t parity,
     return false;
 }
 
+// Wait for completion, ignoring the abort word (draining copies and MMAs).
+__device__ __forceinline__ void quiet_wait(uint32_t bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kWaitLimit && !mbar_test(bar, parity); ++i) {
+    }
+}
+
 // Sequence lengths as the kernel uses them: out-of-range values are clamped.
 __device__ __forceinline__ void seq_shape(const PrefillArgs& a, int cap, int b, int& L, int& n) {
     L = __ldg(a.lens + b);
@@ -139,20 +151,23 @@ __device__ __forceinline__ void seq_shape(const PrefillArgs& a, int cap, int b, 
     n = n < 0 ? 0 : (n > L ? L : n);
 }
 
-// Warp 0: which (sequence, query tile) CTA `i` owns.  Tiles are numbered
-// sequence by sequence, the last (most expensive) tile of a sequence first.
-__device__ void find_tile(const PrefillArgs& a, int cap, int tok_per_tile, int i, int* work) {
+// Warp 0: which (sequence, pair of query tiles) CTA `i` owns.  A sequence with
+// T tiles has ceil(T / 2) items; item k holds tiles T-1-2k and T-2-2k (the last
+// item of an odd count holds tile 0 alone), so the most expensive pair of a
+// sequence gets its lowest CTA index.  work = {b, upper tile}.
+__device__ void find_item(const PrefillArgs& a, int cap, int tok_per_tile, int i, int* work) {
     const int lane = threadIdx.x & 31;
     int base = 0;
     for (int b0 = 0; b0 < a.num_seqs; b0 += 32) {
         const int b = b0 + lane;
-        int nt = 0;
+        int ni = 0, nt = 0;
         if (b < a.num_seqs) {
             int L, n;
             seq_shape(a, cap, b, L, n);
             nt = (n + tok_per_tile - 1) / tok_per_tile;
+            ni = (nt + 1) / 2;
         }
-        int inc = nt;
+        int inc = ni;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int v = __shfl_up_sync(0xffffffffu, inc, o);
@@ -162,29 +177,17 @@ __device__ void find_tile(const PrefillArgs& a, int cap, int tok_per_tile, int i
         if (i < base + total) {
             const unsigned hit = __ballot_sync(0xffffffffu, base + inc > i);
             const int src = __ffs(hit) - 1;
-            const int before = __shfl_sync(0xffffffffu, inc - nt, src);
-            const int count = __shfl_sync(0xffffffffu, nt, src);
+            const int before = __shfl_sync(0xffffffffu, inc - ni, src);
+            const int tiles = __shfl_sync(0xffffffffu, nt, src);
             if (lane == 0) {
                 work[0] = b0 + src;
-                work[1] = count - 1 - (i - base - before);
+                work[1] = tiles - 1 - 2 * (i - base - before);
             }
             return;
         }
         base += total;
     }
     if (lane == 0) work[0] = -1;
-}
-
-// One thread's row of the 128x128 probability tile, K-major and 128B-swizzled:
-// element c of row r sits in half c / 64, 16-byte chunk ((c % 64) / 8) ^ (r % 8).
-__device__ __forceinline__ void store_p_row(uint32_t p_s, int r, const uint32_t (&pk)[64]) {
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-        const uint32_t addr = p_s + (c >> 3) * 16384u + r * 128u + ((((c & 7) ^ (r & 7))) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * c]),
-                     "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
-                     : "memory");
-    }
 }
 
 template <typename T, int D, int BS>
@@ -196,6 +199,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     constexpr uint32_t kIdescS = f16_idesc(kBf16, kPfRows, kPfKv, false);
     constexpr uint32_t kIdescO = f16_idesc(kBf16, kPfRows, D, true);
     static_assert(kPfKv % BS == 0, "a kv tile holds whole blocks");
+    static_assert(D <= 128, "O_t has 128 tensor-memory columns");
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -210,13 +214,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(bar(kBarQ), 1);
         for (int s = 0; s < kPfStages; ++s) {
-            mbar_init(bar(kBarKvFull + s), 1);
-            mbar_init(bar(kBarKvEmpty + s), 1);
+            mbar_init(bar(kBarKFull + s), 1);
+            mbar_init(bar(kBarKEmpty + s), 1);
+            mbar_init(bar(kBarVFull + s), 1);
+            mbar_init(bar(kBarVEmpty + s), 1);
         }
-        mbar_init(bar(kBarSFull), 1);
-        mbar_init(bar(kBarSFull + 1), 1);
-        mbar_init(bar(kBarPFull), 128);
-        mbar_init(bar(kBarODone), 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar(kBarSFull + t), 1);
+            mbar_init(bar(kBarPFull + t), 128);
+            mbar_init(bar(kBarODone + t), 1);
+        }
         mbar_init(bar(kBarDrain), 1);
         misc[1] = 0u;
         fence_mbar_init();
@@ -231,7 +238,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     pdl_wait_primary();
     const int cap = a.max_blocks * BS;
     const int tok_per_tile = kPfRows >> a.log2_group;
-    if (warp == 0) find_tile(a, cap, tok_per_tile, blockIdx.x, work);
+    if (warp == 0) find_item(a, cap, tok_per_tile, blockIdx.x, work);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -239,7 +246,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int b = work[0];
 
     if (b >= 0) {
-        const int qt = work[1];
         const int hk = blockIdx.y;
         const int g = 1 << a.log2_group;
         int L, n;
@@ -251,10 +257,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (n_raw != n) flag(a.err, PKV_DEVERR_BAD_QUERY_COUNT);
         }
         const int q0 = __ldg(a.qstart + b);
-        const int t_lo = qt * tok_per_tile;
-        const int t_hi = min(n, t_lo + tok_per_tile);
-        const int p_hi = L - n + t_hi - 1;  // last query position of the tile
-        const int nkv = p_hi / kPfKv + 1;
+        // tile t covers query tokens [lo_t, hi_t) of the sequence and needs
+        // kv tiles 0 .. nkv_t - 1 (tile 1 the same tiles or one fewer)
+        const int qt0 = work[1];
+        const int lo0 = qt0 * tok_per_tile, hi0 = min(n, lo0 + tok_per_tile);
+        const int lo1 = lo0 - tok_per_tile, hi1 = qt0 > 0 ? lo0 : lo1;
+        const int nkv0 = (L - n + hi0 - 1) / kPfKv + 1;
+        const int nkv1 = qt0 > 0 ? (L - n + hi1 - 1) / kPfKv + 1 : 0;
+        const int nkv = nkv0;
+        const int ntiles = qt0 > 0 ? 2 : 1;
 
         if (warp == 0) {
             // ------------------------------------------------------ producer
@@ -277,161 +288,175 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 return id;
             };
             if (lane == 0) {
-                mbar_arrive_expect_tx(bar(kBarQ), Lay::kTile);
-                tma_load_4d(sb + Lay::kQ, &tq, 0, hk * g, q0 + t_lo, 0, bar(kBarQ));
+                mbar_arrive_expect_tx(bar(kBarQ), ntiles * Lay::kTile);
+                for (int t = 0; t < ntiles; ++t)
+                    tma_load_4d(sb + Lay::kQ + t * Lay::kTile, &tq, 0, hk * g, q0 + (t ? lo1 : lo0),
+                                0, bar(kBarQ));
             }
-            int cur = load_chunk(0), next = 0;
-            int issued = 0;
-            for (int j = 0; j < nkv; ++j) {
+            auto issue = [&](int j, bool is_v, int id) -> bool {
                 const int s = j % kPfStages;
-                if (j % kTilesPerChunk == 0) {
-                    if (j > 0) cur = next;
-                    next = load_chunk(j / kTilesPerChunk + 1);
-                }
+                const int full = (is_v ? kBarVFull : kBarKFull) + s;
+                const int empty = (is_v ? kBarVEmpty : kBarKEmpty) + s;
                 if (j >= kPfStages &&
-                    !warp_wait(bar(kBarKvEmpty + s), ((j / kPfStages) - 1) & 1, abort_word, a.err))
-                    break;
-                const uint32_t ks = sb + Lay::kStage0 + 2u * s * Lay::kTile;
-                const uint32_t vs = ks + Lay::kTile;
-                if (lane == 0) mbar_arrive_expect_tx(bar(kBarKvFull + s), 2u * Lay::kTile);
+                    !warp_wait(bar(empty), ((j / kPfStages) - 1) & 1, abort_word, a.err))
+                    return false;
+                const uint32_t dst = sb + Lay::kStage0 + 2u * s * Lay::kTile + (is_v ? Lay::kTile : 0u);
+                if (lane == 0) mbar_arrive_expect_tx(bar(full), Lay::kTile);
                 __syncwarp();
-                const int id = __shfl_sync(0xffffffffu, cur,
-                                           (j % kTilesPerChunk) * kBlocksPerTile + (lane % kBlocksPerTile));
                 if (lane < kBlocksPerTile) {
                     const int y = (id * a.num_kv_heads + hk) * BS;
 #pragma unroll
-                    for (int h = 0; h < Lay::kHalves; ++h) {
-                        const uint32_t off = h * Lay::kHalfBytes + lane * BS * 128;
-                        tma_load_3d(ks + off, &tk, 0, y, h, bar(kBarKvFull + s));
-                        tma_load_3d(vs + off, &tv, 0, y, h, bar(kBarKvFull + s));
-                    }
+                    for (int h = 0; h < Lay::kHalves; ++h)
+                        tma_load_3d(dst + h * Lay::kHalfBytes + lane * BS * 128, is_v ? &tv : &tk, 0, y,
+                                    h, bar(full));
                 }
-                issued = j + 1;
+                return true;
+            };
+            // K of tile i goes out one step ahead of V of tile i - 1.
+            int cur = load_chunk(0), next = 0;
+            int k_issued = 0, v_issued = 0, id_prev = 0;
+            for (int i = 0; i <= nkv; ++i) {
+                int id = 0;
+                if (i < nkv) {
+                    if (i % kTilesPerChunk == 0) {
+                        if (i > 0) cur = next;
+                        next = load_chunk(i / kTilesPerChunk + 1);
+                    }
+                    id = __shfl_sync(0xffffffffu, cur,
+                                     (i % kTilesPerChunk) * kBlocksPerTile + (lane % kBlocksPerTile));
+                    if (!issue(i, false, id)) break;
+                    k_issued = i + 1;
+                }
+                if (i > 0) {
+                    if (!issue(i - 1, true, id_prev)) break;
+                    v_issued = i;
+                }
+                id_prev = id;
             }
             // Let every copy in flight land before the CTA can exit.
             if (lane == 0) {
-                for (uint32_t i = 0; i < kWaitLimit && !mbar_test(bar(kBarQ), 0); ++i) {
-                }
-                for (int j = issued - kPfStages < 0 ? 0 : issued - kPfStages; j < issued; ++j)
-                    for (uint32_t i = 0;
-                         i < kWaitLimit &&
-                         !mbar_test(bar(kBarKvFull + j % kPfStages), (j / kPfStages) & 1);
-                         ++i) {
-                    }
+                quiet_wait(bar(kBarQ), 0);
+                for (int j = k_issued - kPfStages < 0 ? 0 : k_issued - kPfStages; j < k_issued; ++j)
+                    quiet_wait(bar(kBarKFull + j % kPfStages), (j / kPfStages) & 1);
+                for (int j = v_issued - kPfStages < 0 ? 0 : v_issued - kPfStages; j < v_issued; ++j)
+                    quiet_wait(bar(kBarVFull + j % kPfStages), (j / kPfStages) & 1);
             }
         } else if (warp == 1) {
             // --------------------------------------------------- MMA issuer
             if (lane == 0) {
-                const uint32_t q_s = sb + Lay::kQ, p_s = sb + Lay::kP;
-                auto issue_s = [&](int j) {
+                auto issue_s = [&](int t, int j) {
+                    const uint32_t q_s = sb + Lay::kQ + t * Lay::kTile;
                     const uint32_t ks = sb + Lay::kStage0 + 2u * (j % kPfStages) * Lay::kTile;
-                    const uint32_t dst = tmem + (j & 1) * 128u;
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k) {
                         const uint32_t off = (k >> 2) * 16384u + (k & 3) * 32u;
-                        mma_f16_ss(dst, sw128_desc(q_s + off, 16, 1024),
+                        mma_f16_ss(tmem + 128u * t, sw128_desc(q_s + off, 16, 1024),
                                    sw128_desc(ks + off, 16, 1024), kIdescS, k > 0 ? 1u : 0u);
                     }
-                    mma_commit(bar(kBarSFull + (j & 1)));
+                    mma_commit(bar(kBarSFull + t));
                 };
                 bool ok = one_wait(bar(kBarQ), 0, abort_word, a.err);
-                if (ok) ok = one_wait(bar(kBarKvFull), 0, abort_word, a.err);
+                if (ok) ok = one_wait(bar(kBarKFull), 0, abort_word, a.err);
                 if (ok) {
                     tc_fence_after();
-                    issue_s(0);
+                    for (int t = 0; t < ntiles; ++t) issue_s(t, 0);
+                    mma_commit(bar(kBarKEmpty));
                 }
-                int ev = 0;
                 for (int j = 0; ok && j < nkv; ++j) {
-                    if (j + 1 < nkv) {
-                        const int s1 = (j + 1) % kPfStages;
-                        if (!(ok = one_wait(bar(kBarKvFull + s1), ((j + 1) / kPfStages) & 1,
-                                            abort_word, a.err)))
+                    const uint32_t vs =
+                        sb + Lay::kStage0 + 2u * (j % kPfStages) * Lay::kTile + Lay::kTile;
+                    bool v_ready = false, k_ready = false;
+                    for (int t = 0; ok && t < 2; ++t) {
+                        const int nkv_of_t = t ? nkv1 : nkv0;
+                        if (j >= nkv_of_t) continue;
+                        if (!(ok = one_wait(bar(kBarPFull + t), j & 1, abort_word, a.err))) break;
+                        if (!v_ready && !(ok = one_wait(bar(kBarVFull + j % kPfStages),
+                                                         (j / kPfStages) & 1, abort_word, a.err)))
                             break;
+                        v_ready = true;
                         tc_fence_after();
-                        issue_s(j + 1);
-                    }
-                    const uint32_t vs = sb + Lay::kStage0 + 2u * (j % kPfStages) * Lay::kTile +
-                                        Lay::kTile;
-                    const int parts = j == 0 ? 2 : 1;
-                    for (int part = 0; part < parts; ++part, ++ev) {
-                        if (!(ok = one_wait(bar(kBarPFull), ev & 1, abort_word, a.err))) break;
-                        tc_fence_after();
+                        // P V: P in S_t's columns 0-63 (and, in the first kv
+                        // tile, its rounding residual in columns 64-127)
+                        const int parts = j == 0 ? 2 : 1;
+                        for (int part = 0; part < parts; ++part)
 #pragma unroll
-                        for (int k = 0; k < kPfKv / 16; ++k) {
-                            const uint64_t ad =
-                                sw128_desc(p_s + (k >> 2) * 16384u + (k & 3) * 32u, 16, 1024);
-                            const uint64_t bd = sw128_desc(vs + k * 16 * 128, Lay::kHalfBytes, 1024);
-                            mma_f16_ss(tmem + kTmemO, ad, bd, kIdescO,
-                                       (j > 0 || part > 0 || k > 0) ? 1u : 0u);
+                            for (int k = 0; k < kPfKv / 16; ++k)
+                                mma_f16_ts(tmem + 256u + 128u * t, tmem + 128u * t + 64u * part + 8u * k,
+                                           sw128_desc(vs + k * 16 * 128, Lay::kHalfBytes, 1024), kIdescO,
+                                           (j > 0 || part > 0 || k > 0) ? 1u : 0u);
+                        if (j + 1 == nkv_of_t) mma_commit(bar(kBarODone + t));
+                        if (j + 1 < nkv_of_t) {
+                            if (!k_ready && !(ok = one_wait(bar(kBarKFull + (j + 1) % kPfStages),
+                                                            ((j + 1) / kPfStages) & 1, abort_word,
+                                                            a.err)))
+                                break;
+                            k_ready = true;
+                            tc_fence_after();
+                            issue_s(t, j + 1);
                         }
-                        if (part == parts - 1) mma_commit(bar(kBarKvEmpty + j % kPfStages));
-                        mma_commit(bar(kBarODone));
                     }
+                    if (!ok) break;
+                    mma_commit(bar(kBarVEmpty + j % kPfStages));
+                    if (j + 1 < nkv) mma_commit(bar(kBarKEmpty + (j + 1) % kPfStages));
                 }
                 // Every MMA issued above completes before the tensor memory is freed.
                 mma_commit(bar(kBarDrain));
-                for (uint32_t i = 0; i < kWaitLimit && !mbar_test(bar(kBarDrain), 0); ++i) {
-                }
+                quiet_wait(bar(kBarDrain), 0);
             }
         } else {
             // ------------------------------------------------------ softmax
-            const int quarter = warp & 3;  // the TMEM lane quarter this warp may access
+            const int t = (warp - 2) >> 2;   // query tile of this warpgroup
+            const int quarter = warp & 3;    // the TMEM lane quarter this warp may access
             const int r = quarter * 32 + lane;
             const int tok = r >> a.log2_group;
             const int jh = r & (g - 1);
-            const bool valid = t_lo + tok < t_hi;
+            const int lo_t = t ? lo1 : lo0, hi_t = t ? hi1 : hi0, my_nkv = t ? nkv1 : nkv0;
+            const bool valid = lo_t + tok < hi_t;
             // rows past the sequence's queries reuse the last valid position
-            const int p = L - n + t_lo + min(tok, t_hi - t_lo - 1);
-            const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-            const uint32_t p_s = sb + Lay::kP;
+            const int p = L - n + lo_t + min(tok, hi_t - lo_t - 1);
+            const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+            const uint32_t s_addr = lane_base + 128u * t;
+            const uint32_t o_addr = lane_base + 256u + 128u * t;
             const float sl2 = a.sl2;
             float m_used = -INFINITY, l = 0.f;
-            int ev = 0;
             bool ok = true;
-            for (int j = 0; j < nkv; ++j) {
-                if (!(ok = warp_wait(bar(kBarSFull + (j & 1)), (j >> 1) & 1, abort_word, a.err)))
-                    break;
+            for (int j = 0; j < my_nkv; ++j) {
+                if (!(ok = warp_wait(bar(kBarSFull + t), j & 1, abort_word, a.err))) break;
                 tc_fence_after();
-                uint32_t x[128];
+                uint32_t u[128];
                 {
                     uint32_t c0[32], c1[32], c2[32], c3[32];
-                    const uint32_t src = lane_addr + (j & 1) * 128u;
-                    tmem_ld32(src, c0);
-                    tmem_ld32(src + 32, c1);
-                    tmem_ld32(src + 64, c2);
-                    tmem_ld32(src + 96, c3);
+                    tmem_ld32(s_addr, c0);
+                    tmem_ld32(s_addr + 32, c1);
+                    tmem_ld32(s_addr + 64, c2);
+                    tmem_ld32(s_addr + 96, c3);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        x[i] = c0[i];
-                        x[32 + i] = c1[i];
-                        x[64 + i] = c2[i];
-                        x[96 + i] = c3[i];
+                        u[i] = c0[i];
+                        u[32 + i] = c1[i];
+                        u[64 + i] = c2[i];
+                        u[96 + i] = c3[i];
                     }
                 }
-                // S buffer (j & 1) is free once every lane has read it; the
-                // arrival on P-full below publishes that to the MMA issuer.
                 const int kv0 = j * kPfKv;
+                const int vis = p - kv0;  // columns 0 .. vis are visible to this row
                 float mx[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-                if (kv0 + kPfKv - 1 <= p) {  // the whole tile is visible to this row
+                if (vis >= kPfKv - 1) {
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) {
-                        const float v = __uint_as_float(x[c]) * sl2;
-                        x[c] = __float_as_uint(v);
-                        mx[c & 7] = fmaxf(mx[c & 7], v);
-                    }
+                    for (int c = 0; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(u[c]));
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) {
-                        const float v = kv0 + c <= p ? __uint_as_float(x[c]) * sl2 : -INFINITY;
-                        x[c] = __float_as_uint(v);
-                        mx[c & 7] = fmaxf(mx[c & 7], v);
-                    }
+                    for (int c = 0; c < 128; ++c)
+                        if (c <= vis) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(u[c]));
                 }
-                const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                // maximum of the raw scores, in base-2 units (sl2 > 0; masked
+                // columns never contribute)
+                const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                const float mt = mraw * sl2;
                 const bool rescale = mt > m_used + kRescaleLog2;
                 float factor = 1.f;
                 if (rescale) {
@@ -439,70 +464,73 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     m_used = mt;
                     l *= factor;
                 }
-                uint32_t hi[64], lo[64];
-                float sm[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const float p0 = exp2_approx(__uint_as_float(x[2 * i]) - m_used);
-                    const float p1 = exp2_approx(__uint_as_float(x[2 * i + 1]) - m_used);
-                    sm[i & 3] += p0 + p1;
-                    float r0, r1, q0_, q1_;
-                    hi[i] = Pack<T>::two(p0, p1, r0, r1);
-                    lo[i] = j == 0 ? Pack<T>::two(p0 - r0, p1 - r1, q0_, q1_) : 0u;
-                }
-                l += (sm[0] + sm[1]) + (sm[2] + sm[3]);
-                // The previous P V must be done: it reads the P tile and writes O.
-                if (ev > 0 && !(ok = warp_wait(bar(kBarODone), (ev - 1) & 1, abort_word, a.err)))
-                    break;
-                tc_fence_after();
                 if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+                    // O_t is stable: S_t(j) completing means P_t V(j-1) did too
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t o[32];
-                        tmem_ld32(lane_addr + kTmemO + c * 32, o);
+                        tmem_ld32(o_addr + c * 32, o);
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
                             o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-                        tmem_st32(lane_addr + kTmemO + c * 32, o);
+                        tmem_st32(o_addr + c * 32, o);
                     }
-                    tmem_wait_st();
                 }
-                if (kv0 + kPfKv > L && kv0 + r >= L) {
+                // P = 2^(s sl2 - m) in four chunks of 32 columns; each chunk's
+                // 16 packed pairs go to S_t's columns 16 c .. 16 c + 15 (already
+                // read), the residuals of the first kv tile to 64 + 16 c ..
+                float sm[4] = {0.f, 0.f, 0.f, 0.f};
+                const float nm = -m_used;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t hi[16], lo[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int c0 = 32 * c + 2 * i;
+                        const float p0 = c0 <= vis ? exp2_approx(fmaf(__uint_as_float(u[c0]), sl2, nm)) : 0.f;
+                        const float p1 =
+                            c0 + 1 <= vis ? exp2_approx(fmaf(__uint_as_float(u[c0 + 1]), sl2, nm)) : 0.f;
+                        sm[i & 3] += p0 + p1;
+                        float r0, r1, z0, z1;
+                        hi[i] = Pack<T>::two(p0, p1, r0, r1);
+                        lo[i] = Pack<T>::two(p0 - r0, p1 - r1, z0, z1);
+                    }
+                    tmem_st16(s_addr + 16 * c, hi);
+                    if (j == 0) tmem_st16(s_addr + 64 + 16 * c, lo);
+                }
+                l += (sm[0] + sm[1]) + (sm[2] + sm[3]);
+                if (t == 0 && kv0 + kPfKv > L) {
                     // Past the context the slots hold whatever a block holds
                     // (possibly NaN or Inf); P is 0 there, but 0 * NaN is NaN, so
-                    // the V rows are zeroed.  The copies landed before S_j was
-                    // computed, and nothing reads this stage until P V_j.
-                    const uint32_t vrow =
-                        sb + Lay::kStage0 + 2u * (j % kPfStages) * Lay::kTile + Lay::kTile + r * 128u;
+                    // tile 0's warps zero those V rows once the copy has landed
+                    // (tile 0 sees every kv tile tile 1 does, and its P V is
+                    // issued first).
+                    if (!(ok = warp_wait(bar(kBarVFull + j % kPfStages), (j / kPfStages) & 1,
+                                         abort_word, a.err)))
+                        break;
+                    if (kv0 + r >= L) {
+                        const uint32_t vrow = sb + Lay::kStage0 + 2u * (j % kPfStages) * Lay::kTile +
+                                              Lay::kTile + r * 128u;
 #pragma unroll
-                    for (int h = 0; h < Lay::kHalves; ++h)
+                        for (int h = 0; h < Lay::kHalves; ++h)
 #pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(
-                                             vrow + h * Lay::kHalfBytes + c * 16),
-                                         "r"(0u)
-                                         : "memory");
-                }
-                store_p_row(p_s, r, hi);
-                fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive(bar(kBarPFull));
-                ++ev;
-                if (j == 0) {
-                    // second product of tile 0: the rounding residual of P
-                    if (!(ok = warp_wait(bar(kBarODone), (ev - 1) & 1, abort_word, a.err))) break;
-                    store_p_row(p_s, r, lo);
+                            for (int c = 0; c < 8; ++c)
+                                asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(
+                                                 vrow + h * Lay::kHalfBytes + c * 16),
+                                             "r"(0u)
+                                             : "memory");
+                    }
                     fence_proxy_async_smem();
-                    tc_fence_before();
-                    mbar_arrive(bar(kBarPFull));
-                    ++ev;
                 }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(kBarPFull + t));
             }
-            if (ok && ev > 0) ok = warp_wait(bar(kBarODone), (ev - 1) & 1, abort_word, a.err);
-            if (ok) {
+            if (ok && my_nkv > 0) ok = warp_wait(bar(kBarODone + t), 0, abort_word, a.err);
+            if (ok && my_nkv > 0) {
                 tc_fence_after();
-                const int64_t qrow = static_cast<int64_t>(q0) + t_lo + tok;
+                const int64_t qrow = static_cast<int64_t>(q0) + lo_t + tok;
                 const bool store = valid && qrow >= 0 && qrow < a.num_tokens;
                 if (valid && !store) flag(a.err, PKV_DEVERR_BAD_QUERY_COUNT);
                 const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -511,7 +539,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
-                    tmem_ld32(lane_addr + kTmemO + c * 32, o);
+                    tmem_ld32(o_addr + c * 32, o);
                     tmem_wait_ld();
                     uint32_t pk[16];
 #pragma unroll
@@ -591,8 +619,9 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
     auto* k = prefill_kernel<T, D, BS>;
     cudaError_t e = opt_in_smem<PrefillTag<T, D, BS>>(reinterpret_cast<const void*>(k));
     if (e != cudaSuccess) return e;
+    // items per sequence = ceil(ceil(n / tpt) / 2) <= n / (2 tpt) + 1
     const int tok_per_tile = kPfRows >> a.log2_group;
-    dim3 grid(static_cast<unsigned>(a.num_tokens / tok_per_tile + a.num_seqs),
+    dim3 grid(static_cast<unsigned>(a.num_tokens / (2 * tok_per_tile) + a.num_seqs),
               static_cast<unsigned>(a.num_kv_heads));
     return launch_dependent(k, grid, dim3(kPfThreads), PfLayout<D>::kAlloc, stream, tq, tk, tv, a);
 }
