@@ -101,21 +101,33 @@ struct PrefillArgs {
     float sl2;  // scale * log2(e)
 };
 
+// Two floats rounded to one 32-bit pair of T (first in the low half).
+template <typename T>
+__device__ __forceinline__ uint32_t pack_pair(float lo, float hi) {
+    float r0, r1;
+    return Pack<T>::two(lo, hi, r0, r1);
+}
+
 __device__ __forceinline__ void flag(int32_t* err, int bit) {
     if (err) atomicOr(err, bit);
 }
 
-// Bounded wait that also gives up when another role raised the abort word.
+// Every wait below gives up after kWaitCycles SM cycles (about half a second):
+// a protocol fault then costs each CTA a bounded delay, never a hang.
+constexpr long long kWaitCycles = 1ll << 30;
+
+// Wait that also gives up when another role raised the abort word.
 // Warp-uniform: every lane of the calling warp must call it.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
                                           volatile uint32_t* abort_word, int32_t* err) {
     bool ok = false;
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    const long long t0 = clock64();
+    for (;;) {
         if (mbar_test(bar, parity)) {
             ok = true;
             break;
         }
-        if (*abort_word) break;
+        if (*abort_word || clock64() - t0 > kWaitCycles) break;
     }
     ok = __all_sync(0xffffffffu, ok);
     if (!ok && *abort_word == 0u) {
@@ -128,9 +140,11 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
 // Single-thread variant (MMA issuer).
 __device__ __forceinline__ bool one_wait(uint32_t bar, uint32_t parity,
                                          volatile uint32_t* abort_word, int32_t* err) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    const long long t0 = clock64();
+    for (;;) {
         if (mbar_test(bar, parity)) return true;
         if (*abort_word) return false;
+        if (clock64() - t0 > kWaitCycles) break;
     }
     *abort_word = 1u;
     flag(err, PKV_DEVERR_WAIT_TIMEOUT);
@@ -139,7 +153,8 @@ __device__ __forceinline__ bool one_wait(uint32_t bar, uint32_t parity,
 
 // Wait for completion, ignoring the abort word (draining copies and MMAs).
 __device__ __forceinline__ void quiet_wait(uint32_t bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitLimit && !mbar_test(bar, parity); ++i) {
+    const long long t0 = clock64();
+    while (!mbar_test(bar, parity) && clock64() - t0 <= kWaitCycles) {
     }
 }
 
@@ -482,22 +497,43 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 // read), the residuals of the first kv tile to 64 + 16 c ..
                 float sm[4] = {0.f, 0.f, 0.f, 0.f};
                 const float nm = -m_used;
+                // The path must be the same for the whole warp: the TMEM stores
+                // below are warp-collective.
+                if (j == 0 || __any_sync(0xffffffffu, vis < kPfKv - 1)) {
+                    // masked tile (and, in the first kv tile, the residuals)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t hi[16], lo[16];
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t hi[16], lo[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int c0 = 32 * c + 2 * i;
-                        const float p0 = c0 <= vis ? exp2_approx(fmaf(__uint_as_float(u[c0]), sl2, nm)) : 0.f;
-                        const float p1 =
-                            c0 + 1 <= vis ? exp2_approx(fmaf(__uint_as_float(u[c0 + 1]), sl2, nm)) : 0.f;
-                        sm[i & 3] += p0 + p1;
-                        float r0, r1, z0, z1;
-                        hi[i] = Pack<T>::two(p0, p1, r0, r1);
-                        lo[i] = Pack<T>::two(p0 - r0, p1 - r1, z0, z1);
+                        for (int i = 0; i < 16; ++i) {
+                            const int c0 = 32 * c + 2 * i;
+                            const float p0 =
+                                c0 <= vis ? exp2_approx(fmaf(__uint_as_float(u[c0]), sl2, nm)) : 0.f;
+                            const float p1 =
+                                c0 + 1 <= vis ? exp2_approx(fmaf(__uint_as_float(u[c0 + 1]), sl2, nm)) : 0.f;
+                            sm[i & 3] += p0 + p1;
+                            float r0, r1, z0, z1;
+                            hi[i] = Pack<T>::two(p0, p1, r0, r1);
+                            lo[i] = Pack<T>::two(p0 - r0, p1 - r1, z0, z1);
+                        }
+                        tmem_st16(s_addr + 16 * c, hi);
+                        if (j == 0) tmem_st16(s_addr + 64 + 16 * c, lo);
                     }
-                    tmem_st16(s_addr + 16 * c, hi);
-                    if (j == 0) tmem_st16(s_addr + 64 + 16 * c, lo);
+                } else {
+                    // every column visible, rounded P only
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t hi[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int c0 = 32 * c + 2 * i;
+                            const float p0 = exp2_approx(fmaf(__uint_as_float(u[c0]), sl2, nm));
+                            const float p1 = exp2_approx(fmaf(__uint_as_float(u[c0 + 1]), sl2, nm));
+                            sm[i & 3] += p0 + p1;
+                            hi[i] = pack_pair<T>(p0, p1);
+                        }
+                        tmem_st16(s_addr + 16 * c, hi);
+                    }
                 }
                 l += (sm[0] + sm[1]) + (sm[2] + sm[3]);
                 if (t == 0 && kv0 + kPfKv > L) {
