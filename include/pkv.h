@@ -204,9 +204,9 @@ pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* out, const v
  * a single decode token, n_b = 0 nothing.
  * Arithmetic: fp16/bf16 inputs; Q K^T and P V on the tensor cores with fp32
  * accumulation; softmax in fp32 (base 2, scale * log2 e folded in); the
- * probabilities enter P V rounded to `dtype`, except in the first 128-token
- * tile of every sequence, where their rounding residual is added by a second
- * product; output rounded to `dtype`.
+ * probabilities enter P V rounded to `dtype` (for query rows that see at most
+ * 128 tokens their rounding residual is added by a second product); output
+ * rounded to `dtype`.  scale must be positive.
  *   out, q          device [num_tokens][num_heads][head_dim], 16-byte aligned;
  *                   rows of a sequence are consecutive, sequences in order.
  *   k_cache, v_cache device pools, 16-byte aligned (read only).

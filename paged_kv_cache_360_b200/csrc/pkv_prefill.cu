@@ -11,18 +11,19 @@
 // head) -- tile 0 the later one, tile 1 the one before it -- against the same
 // stream of 128-token kv tiles, so each K/V tile is loaded once for 256 rows and
 // the tensor core alternates between the tiles while each tile's softmax runs:
-//   warp 0      producer: both Q tiles (4-D TMA boxes), then per kv tile one
+//   warp 8      producer: both Q tiles (4-D TMA boxes), then per kv tile one
 //               3-D TMA box per (block, 64-column half) of K and of V into two
 //               2-stage rings (K freed by Q K^T, V by P V), K one tile ahead;
-//   warp 1      MMA issuer (one thread) and tensor-memory owner.  Per tile t:
+//   warp 9      MMA issuer (one thread) and tensor-memory owner.  Per tile t:
 //               S_t = Q_t K_j^T (fp32, 128 TMEM columns), then O_t += P_t V_j
 //               with P_t read from tensor memory, O_t in its own 128 columns;
 //               order: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ...
-//   warps 2-5   softmax of tile 0, warps 6-9 of tile 1; one row per thread
+//   warps 0-3   softmax of tile 0, warps 4-7 of tile 1; one row per thread
 //               (TMEM lane = row): causal mask, running maximum, P = 2^(s - m)
 //               rounded to the input type and written back over S's first 64
-//               columns; in a sequence's first kv tile the rounding residual
-//               goes to columns 64-127 and enters P V as a second product.  O is
+//               columns; for rows that see only the first kv tile the
+//               rounding residual goes to columns 64-127 and enters P V as a
+//               second product.  O is
 //               rescaled in tensor memory only when the maximum grows by more
 //               than 2^8.  The MMAs of one thread complete in issue order, so
 //               when S_t(j) is complete so is P_t V(j-1): O_t is stable during
@@ -50,12 +51,21 @@
 namespace pkv {
 namespace {
 
-constexpr int kPfThreads = 320;      // producer warp, MMA warp, 2 softmax warpgroups
+constexpr int kPfThreads = 384;      // 2 softmax warpgroups, then producer, MMA, 2 idle warps
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+// Register split (setmaxnreg): the launch gives 384 threads x 168 registers =
+// 64512; the softmax warpgroups take 224 each, the third warpgroup 56:
+// 256 x 224 + 128 x 56 = 64512.
+constexpr int kSoftmaxRegs = 224;
+constexpr int kOtherRegs = 56;
+static_assert(256 * kSoftmaxRegs + 128 * kOtherRegs <= kPfThreads * 168, "register split");
 constexpr int kPfRows = 128;         // MMA M: query rows per tile
 constexpr int kPfKv = 128;           // kv tokens per tile: N of Q K^T, K of P V
 constexpr int kPfStages = 2;         // K and V ring depth
 constexpr uint32_t kTmemCols = 512;  // S_t at 128 t, O_t at 256 + 128 t
 constexpr float kRescaleLog2 = 8.f;  // rescale O when the maximum grows by > 2^8
+constexpr int kResidualTiles = 1;    // P's rounding residual for rows inside the first kv tile
 
 enum : int {
     kBarQ = 0,
@@ -100,6 +110,39 @@ struct PrefillArgs {
     int32_t num_blocks;
     float sl2;  // scale * log2(e)
 };
+
+// Paired fp32 arithmetic (two lanes per 64-bit register) and a 3-input max.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t r, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+                     taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                 "r"(r[7])
+                 : "memory");
+}
 
 // Two floats rounded to one 32-bit pair of T (first in the low half).
 template <typename T>
@@ -246,24 +289,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         prefetch_tensormap(&tk);
         prefetch_tensormap(&tv);
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(sb + Lay::kMisc, kTmemCols);
         tmem_relinquish();
     }
     pdl_wait_primary();
     const int cap = a.max_blocks * BS;
     const int tok_per_tile = kPfRows >> a.log2_group;
-    if (warp == 0) find_item(a, cap, tok_per_tile, blockIdx.x, work);
+    if (warp == kProducerWarp) find_item(a, cap, tok_per_tile, blockIdx.x, work);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
     const int b = work[0];
-
+    const int hk = blockIdx.y;
+    const int g = 1 << a.log2_group;
+    int L = 0, n = 0, q0 = 0, qt0 = 0;
     if (b >= 0) {
-        const int hk = blockIdx.y;
-        const int g = 1 << a.log2_group;
-        int L, n;
         seq_shape(a, cap, b, L, n);
         if (threadIdx.x == 0) {
             const int L_raw = __ldg(a.lens + b);
@@ -271,18 +313,213 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (L_raw != L) flag(a.err, PKV_DEVERR_BAD_CONTEXT_LEN);
             if (n_raw != n) flag(a.err, PKV_DEVERR_BAD_QUERY_COUNT);
         }
-        const int q0 = __ldg(a.qstart + b);
-        // tile t covers query tokens [lo_t, hi_t) of the sequence and needs
-        // kv tiles 0 .. nkv_t - 1 (tile 1 the same tiles or one fewer)
-        const int qt0 = work[1];
-        const int lo0 = qt0 * tok_per_tile, hi0 = min(n, lo0 + tok_per_tile);
-        const int lo1 = lo0 - tok_per_tile, hi1 = qt0 > 0 ? lo0 : lo1;
-        const int nkv0 = (L - n + hi0 - 1) / kPfKv + 1;
-        const int nkv1 = qt0 > 0 ? (L - n + hi1 - 1) / kPfKv + 1 : 0;
-        const int nkv = nkv0;
-        const int ntiles = qt0 > 0 ? 2 : 1;
+        q0 = __ldg(a.qstart + b);
+        qt0 = work[1];
+    }
+    // tile t covers query tokens [lo_t, hi_t) of the sequence and needs kv
+    // tiles 0 .. nkv_t - 1 (tile 1 the same tiles or one fewer)
+    const int lo0 = qt0 * tok_per_tile, hi0 = min(n, lo0 + tok_per_tile);
+    const int lo1 = lo0 - tok_per_tile, hi1 = qt0 > 0 ? lo0 : lo1;
+    const int nkv0 = (L - n + hi0 - 1) / kPfKv + 1;
+    const int nkv1 = qt0 > 0 ? (L - n + hi1 - 1) / kPfKv + 1 : 0;
+    const int nkv = nkv0;
+    const int ntiles = qt0 > 0 ? 2 : 1;
 
-        if (warp == 0) {
+    // Each role raises or lowers its register budget first thing in its own
+    // branch, so the compiler gives each region the matching limit.
+    if (warp < 8) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+        if (b >= 0) {
+            // ------------------------------------------------------ softmax
+            const int t = warp >> 2;         // query tile of this warpgroup
+            const int quarter = warp & 3;    // the TMEM lane quarter this warp may access
+            const int r = quarter * 32 + lane;
+            const int tok = r >> a.log2_group;
+            const int jh = r & (g - 1);
+            const int lo_t = t ? lo1 : lo0, hi_t = t ? hi1 : hi0, my_nkv = t ? nkv1 : nkv0;
+            const bool valid = lo_t + tok < hi_t;
+            // rows past the sequence's queries reuse the last valid position
+            const int p = L - n + lo_t + min(tok, hi_t - lo_t - 1);
+            const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+            const uint32_t s_addr = lane_base + 128u * t;
+            const uint32_t o_addr = lane_base + 256u + 128u * t;
+            const float sl2 = a.sl2;
+            float m_used = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int j = 0; j < my_nkv; ++j) {
+                if (!(ok = warp_wait(bar(kBarSFull + t), j & 1, abort_word, a.err))) break;
+                tc_fence_after();
+                uint32_t u[128];
+                {
+                    uint32_t c0[32], c1[32], c2[32], c3[32];
+                    tmem_ld32(s_addr, c0);
+                    tmem_ld32(s_addr + 32, c1);
+                    tmem_ld32(s_addr + 64, c2);
+                    tmem_ld32(s_addr + 96, c3);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        u[i] = c0[i];
+                        u[32 + i] = c1[i];
+                        u[64 + i] = c2[i];
+                        u[96 + i] = c3[i];
+                    }
+                }
+                const int kv0 = j * kPfKv;
+                const int vis = p - kv0;  // columns 0 .. vis are visible to this row
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                if (__any_sync(0xffffffffu, vis < kPfKv - 1)) {
+                    // diagonal tile: masked scores become -inf here (whatever the
+                    // slot held), so that 2^(-inf) = 0 below needs no select
+#pragma unroll
+                    for (int c = 0; c < 128; c += 2) {
+                        const float v0 = c <= vis ? __uint_as_float(u[c]) : -INFINITY;
+                        const float v1 = c + 1 <= vis ? __uint_as_float(u[c + 1]) : -INFINITY;
+                        u[c] = __float_as_uint(v0);
+                        u[c + 1] = __float_as_uint(v1);
+                        mx[(c >> 1) & 3] = max3(mx[(c >> 1) & 3], v0, v1);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 128; c += 2)
+                        mx[(c >> 1) & 3] = max3(mx[(c >> 1) & 3], __uint_as_float(u[c]),
+                                                __uint_as_float(u[c + 1]));
+                }
+                // maximum of the raw scores, in base-2 units (sl2 > 0; masked
+                // columns never contribute)
+                const float mraw = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                const float mt = mraw * sl2;
+                const bool rescale = mt > m_used + kRescaleLog2;
+                float factor = 1.f;
+                if (rescale) {
+                    factor = exp2_approx(m_used - mt);
+                    m_used = mt;
+                    l *= factor;
+                }
+                if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+                    // O_t is stable: S_t(j) completing means P_t V(j-1) did too
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(o_addr + c * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+                        tmem_st32(o_addr + c * 32, o);
+                    }
+                }
+                // P = 2^(s sl2 - m), 16 columns at a time: the 8 packed pairs go
+                // to S_t's columns 8 k .. 8 k + 7 (those scores are already in
+                // registers).  Paired fp32 arithmetic for the scaling and sums.
+                const uint64_t s2 = f2(sl2, sl2), n2 = f2(-m_used, -m_used);
+                uint64_t acc[2] = {0ull, 0ull};
+                // Rows that see at most kResidualTiles kv tiles also send the
+                // first tile's rounding residual P - round(P) to columns 64 + 8 k
+                // (with few visible tokens the 2^-9 relative rounding of each
+                // weight does not average out).  Warp-uniform, like the stores.
+                if (j == 0 && my_nkv <= kResidualTiles) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        uint32_t pk[8], rk[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int c0 = 16 * k + 2 * i;
+                            float x0, x1;
+                            f2_split(ffma2(f2(__uint_as_float(u[c0]), __uint_as_float(u[c0 + 1])), s2,
+                                           n2),
+                                     x0, x1);
+                            const float p0 = exp2_approx(x0), p1 = exp2_approx(x1);
+                            acc[i & 1] = fadd2(acc[i & 1], f2(p0, p1));
+                            float r0, r1, z0, z1;
+                            pk[i] = Pack<T>::two(p0, p1, r0, r1);
+                            rk[i] = Pack<T>::two(p0 - r0, p1 - r1, z0, z1);
+                        }
+                        tmem_st8(s_addr + 8 * k, pk);
+                        tmem_st8(s_addr + 64 + 8 * k, rk);
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int c0 = 16 * k + 2 * i;
+                            float x0, x1;
+                            f2_split(ffma2(f2(__uint_as_float(u[c0]), __uint_as_float(u[c0 + 1])), s2,
+                                           n2),
+                                     x0, x1);
+                            const float p0 = exp2_approx(x0), p1 = exp2_approx(x1);
+                            acc[i & 1] = fadd2(acc[i & 1], f2(p0, p1));
+                            pk[i] = pack_pair<T>(p0, p1);
+                        }
+                        tmem_st8(s_addr + 8 * k, pk);
+                    }
+                }
+                float sa, sb_, sc, sd;
+                f2_split(acc[0], sa, sb_);
+                f2_split(acc[1], sc, sd);
+                l += (sa + sb_) + (sc + sd);
+                if (t == 0 && kv0 + kPfKv > L) {
+                    // Past the context the slots hold whatever a block holds
+                    // (possibly NaN or Inf); P is 0 there, but 0 * NaN is NaN, so
+                    // tile 0's warps zero those V rows once the copy has landed
+                    // (tile 0 sees every kv tile tile 1 does, and its P V is
+                    // issued first).
+                    if (!(ok = warp_wait(bar(kBarVFull + j % kPfStages), (j / kPfStages) & 1,
+                                         abort_word, a.err)))
+                        break;
+                    if (kv0 + r >= L) {
+                        const uint32_t vrow = sb + Lay::kStage0 + 2u * (j % kPfStages) * Lay::kTile +
+                                              Lay::kTile + r * 128u;
+#pragma unroll
+                        for (int h = 0; h < Lay::kHalves; ++h)
+#pragma unroll
+                            for (int c = 0; c < 8; ++c)
+                                asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(
+                                                 vrow + h * Lay::kHalfBytes + c * 16),
+                                             "r"(0u)
+                                             : "memory");
+                    }
+                    fence_proxy_async_smem();
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(kBarPFull + t));
+            }
+            if (ok && my_nkv > 0) ok = warp_wait(bar(kBarODone + t), 0, abort_word, a.err);
+            if (ok && my_nkv > 0) {
+                tc_fence_after();
+                const int64_t qrow = static_cast<int64_t>(q0) + lo_t + tok;
+                const bool store = valid && qrow >= 0 && qrow < a.num_tokens;
+                if (valid && !store) flag(a.err, PKV_DEVERR_BAD_QUERY_COUNT);
+                const float inv = l > 0.f ? 1.f / l : 0.f;
+                T* dst = static_cast<T*>(a.out) +
+                         (qrow * a.num_heads + static_cast<int64_t>(hk) * g + jh) * D;
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + c * 32, o);
+                    tmem_wait_ld();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float r0, r1;
+                        pk[i] = Pack<T>::two(__uint_as_float(o[2 * i]) * inv,
+                                             __uint_as_float(o[2 * i + 1]) * inv, r0, r1);
+                    }
+                    if (store) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                }
+            }
+        }
+    } else {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
+        if (b >= 0 && warp == kProducerWarp) {
             // ------------------------------------------------------ producer
             // Table entries come 32 at a time (one per lane, one coalesced
             // load), the next 32 prefetched while the current ones are used;
@@ -356,7 +593,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 for (int j = v_issued - kPfStages < 0 ? 0 : v_issued - kPfStages; j < v_issued; ++j)
                     quiet_wait(bar(kBarVFull + j % kPfStages), (j / kPfStages) & 1);
             }
-        } else if (warp == 1) {
+        } else if (b >= 0 && warp == kMmaWarp) {
             // --------------------------------------------------- MMA issuer
             if (lane == 0) {
                 auto issue_s = [&](int t, int j) {
@@ -392,7 +629,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         tc_fence_after();
                         // P V: P in S_t's columns 0-63 (and, in the first kv
                         // tile, its rounding residual in columns 64-127)
-                        const int parts = j == 0 ? 2 : 1;
+                        const int parts = (j == 0 && nkv_of_t <= kResidualTiles) ? 2 : 1;
                         for (int part = 0; part < parts; ++part)
 #pragma unroll
                             for (int k = 0; k < kPfKv / 16; ++k)
@@ -418,185 +655,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 mma_commit(bar(kBarDrain));
                 quiet_wait(bar(kBarDrain), 0);
             }
-        } else {
-            // ------------------------------------------------------ softmax
-            const int t = (warp - 2) >> 2;   // query tile of this warpgroup
-            const int quarter = warp & 3;    // the TMEM lane quarter this warp may access
-            const int r = quarter * 32 + lane;
-            const int tok = r >> a.log2_group;
-            const int jh = r & (g - 1);
-            const int lo_t = t ? lo1 : lo0, hi_t = t ? hi1 : hi0, my_nkv = t ? nkv1 : nkv0;
-            const bool valid = lo_t + tok < hi_t;
-            // rows past the sequence's queries reuse the last valid position
-            const int p = L - n + lo_t + min(tok, hi_t - lo_t - 1);
-            const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-            const uint32_t s_addr = lane_base + 128u * t;
-            const uint32_t o_addr = lane_base + 256u + 128u * t;
-            const float sl2 = a.sl2;
-            float m_used = -INFINITY, l = 0.f;
-            bool ok = true;
-            for (int j = 0; j < my_nkv; ++j) {
-                if (!(ok = warp_wait(bar(kBarSFull + t), j & 1, abort_word, a.err))) break;
-                tc_fence_after();
-                uint32_t u[128];
-                {
-                    uint32_t c0[32], c1[32], c2[32], c3[32];
-                    tmem_ld32(s_addr, c0);
-                    tmem_ld32(s_addr + 32, c1);
-                    tmem_ld32(s_addr + 64, c2);
-                    tmem_ld32(s_addr + 96, c3);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        u[i] = c0[i];
-                        u[32 + i] = c1[i];
-                        u[64 + i] = c2[i];
-                        u[96 + i] = c3[i];
-                    }
-                }
-                const int kv0 = j * kPfKv;
-                const int vis = p - kv0;  // columns 0 .. vis are visible to this row
-                float mx[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-                if (vis >= kPfKv - 1) {
-#pragma unroll
-                    for (int c = 0; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(u[c]));
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 128; ++c)
-                        if (c <= vis) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(u[c]));
-                }
-                // maximum of the raw scores, in base-2 units (sl2 > 0; masked
-                // columns never contribute)
-                const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-                const float mt = mraw * sl2;
-                const bool rescale = mt > m_used + kRescaleLog2;
-                float factor = 1.f;
-                if (rescale) {
-                    factor = exp2_approx(m_used - mt);
-                    m_used = mt;
-                    l *= factor;
-                }
-                if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-                    // O_t is stable: S_t(j) completing means P_t V(j-1) did too
-#pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(o_addr + c * 32, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-                        tmem_st32(o_addr + c * 32, o);
-                    }
-                }
-                // P = 2^(s sl2 - m) in four chunks of 32 columns; each chunk's
-                // 16 packed pairs go to S_t's columns 16 c .. 16 c + 15 (already
-                // read), the residuals of the first kv tile to 64 + 16 c ..
-                float sm[4] = {0.f, 0.f, 0.f, 0.f};
-                const float nm = -m_used;
-                // The path must be the same for the whole warp: the TMEM stores
-                // below are warp-collective.
-                if (j == 0 || __any_sync(0xffffffffu, vis < kPfKv - 1)) {
-                    // masked tile (and, in the first kv tile, the residuals)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t hi[16], lo[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int c0 = 32 * c + 2 * i;
-                            const float p0 =
-                                c0 <= vis ? exp2_approx(fmaf(__uint_as_float(u[c0]), sl2, nm)) : 0.f;
-                            const float p1 =
-                                c0 + 1 <= vis ? exp2_approx(fmaf(__uint_as_float(u[c0 + 1]), sl2, nm)) : 0.f;
-                            sm[i & 3] += p0 + p1;
-                            float r0, r1, z0, z1;
-                            hi[i] = Pack<T>::two(p0, p1, r0, r1);
-                            lo[i] = Pack<T>::two(p0 - r0, p1 - r1, z0, z1);
-                        }
-                        tmem_st16(s_addr + 16 * c, hi);
-                        if (j == 0) tmem_st16(s_addr + 64 + 16 * c, lo);
-                    }
-                } else {
-                    // every column visible, rounded P only
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t hi[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int c0 = 32 * c + 2 * i;
-                            const float p0 = exp2_approx(fmaf(__uint_as_float(u[c0]), sl2, nm));
-                            const float p1 = exp2_approx(fmaf(__uint_as_float(u[c0 + 1]), sl2, nm));
-                            sm[i & 3] += p0 + p1;
-                            hi[i] = pack_pair<T>(p0, p1);
-                        }
-                        tmem_st16(s_addr + 16 * c, hi);
-                    }
-                }
-                l += (sm[0] + sm[1]) + (sm[2] + sm[3]);
-                if (t == 0 && kv0 + kPfKv > L) {
-                    // Past the context the slots hold whatever a block holds
-                    // (possibly NaN or Inf); P is 0 there, but 0 * NaN is NaN, so
-                    // tile 0's warps zero those V rows once the copy has landed
-                    // (tile 0 sees every kv tile tile 1 does, and its P V is
-                    // issued first).
-                    if (!(ok = warp_wait(bar(kBarVFull + j % kPfStages), (j / kPfStages) & 1,
-                                         abort_word, a.err)))
-                        break;
-                    if (kv0 + r >= L) {
-                        const uint32_t vrow = sb + Lay::kStage0 + 2u * (j % kPfStages) * Lay::kTile +
-                                              Lay::kTile + r * 128u;
-#pragma unroll
-                        for (int h = 0; h < Lay::kHalves; ++h)
-#pragma unroll
-                            for (int c = 0; c < 8; ++c)
-                                asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(
-                                                 vrow + h * Lay::kHalfBytes + c * 16),
-                                             "r"(0u)
-                                             : "memory");
-                    }
-                    fence_proxy_async_smem();
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar(kBarPFull + t));
-            }
-            if (ok && my_nkv > 0) ok = warp_wait(bar(kBarODone + t), 0, abort_word, a.err);
-            if (ok && my_nkv > 0) {
-                tc_fence_after();
-                const int64_t qrow = static_cast<int64_t>(q0) + lo_t + tok;
-                const bool store = valid && qrow >= 0 && qrow < a.num_tokens;
-                if (valid && !store) flag(a.err, PKV_DEVERR_BAD_QUERY_COUNT);
-                const float inv = l > 0.f ? 1.f / l : 0.f;
-                T* dst = static_cast<T*>(a.out) +
-                         (qrow * a.num_heads + static_cast<int64_t>(hk) * g + jh) * D;
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(o_addr + c * 32, o);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float r0, r1;
-                        pk[i] = Pack<T>::two(__uint_as_float(o[2 * i]) * inv,
-                                             __uint_as_float(o[2 * i + 1]) * inv, r0, r1);
-                    }
-                    if (store) {
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                    }
-                }
-            }
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -693,8 +756,8 @@ extern "C" pkv_status paged_attention_prefill(const pkv_cache_desc* desc, void* 
     const int g = num_heads / desc->num_kv_heads;
     if ((g & (g - 1)) != 0 || g > kPfRows)
         return fail(PKV_ERR_UNSUPPORTED, "num_heads / num_kv_heads must be a power of two <= 128");
-    if (!(scale == scale) || scale == INFINITY || scale == -INFINITY)
-        return fail(PKV_ERR_INVALID_ARG, "scale must be finite");
+    if (!(scale > 0.f) || scale == INFINITY)
+        return fail(PKV_ERR_INVALID_ARG, "scale must be positive and finite");
     if (static_cast<int64_t>(max_blocks_per_seq) * desc->block_size > INT32_MAX / 2)
         return fail(PKV_ERR_UNSUPPORTED, "max_blocks_per_seq * block_size too large");
     if (num_tokens == 0 || num_seqs == 0) return PKV_OK;

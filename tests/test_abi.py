@@ -123,6 +123,7 @@ def test_prefill_rejects_bad_arguments(lib):
     assert _prefill(lib, d, H=6) == 2                    # group 3: not a power of two
     assert _prefill(lib, d, H=2 * 256) == 2              # group 256 > 128
     assert _prefill(lib, d, scale=float("inf")) == 1
+    assert _prefill(lib, d, scale=-0.1) == 1
     assert _prefill(lib, d, T=-1) == 1
     assert _prefill(lib, d, mb=0) == 1
     assert _prefill(lib, d, qs=None) == 1
