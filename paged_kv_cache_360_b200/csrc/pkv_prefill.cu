@@ -350,21 +350,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 if (!(ok = warp_wait(bar(kBarSFull + t), j & 1, abort_word, a.err))) break;
                 tc_fence_after();
                 uint32_t u[128];
-                {
-                    uint32_t c0[32], c1[32], c2[32], c3[32];
-                    tmem_ld32(s_addr, c0);
-                    tmem_ld32(s_addr + 32, c1);
-                    tmem_ld32(s_addr + 64, c2);
-                    tmem_ld32(s_addr + 96, c3);
-                    tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        u[i] = c0[i];
-                        u[32 + i] = c1[i];
-                        u[64 + i] = c2[i];
-                        u[96 + i] = c3[i];
-                    }
-                }
+                for (int c = 0; c < 4; ++c)
+                    tmem_ld32(s_addr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(u + 32 * c));
+                tmem_wait_ld();
                 const int kv0 = j * kPfKv;
                 const int vis = p - kv0;  // columns 0 .. vis are visible to this row
                 float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
