@@ -64,3 +64,16 @@ def compare(gpu_out, ref, seqs=None, what=""):
 
 def words(t):
     return oracle.words(t)
+
+
+def prefix_rows(tokens, Hkv, D, dtype):
+    """K and V rows [len, Hkv, D] where the row at position p depends only on
+    tokens[:p + 1] -- as a model's keys and values do, so that requests with the
+    same prompt prefix have the same rows there."""
+    from paged_kv_cache_360_b200.workloads import normal_tensor
+    ks, vs = [], []
+    for p in range(len(tokens)):
+        rng = np.random.default_rng([7] + [int(t) for t in tokens[:p + 1]])
+        ks.append(normal_tensor(rng, (Hkv, D), dtype))
+        vs.append(normal_tensor(rng, (Hkv, D), dtype))
+    return torch.stack(ks), torch.stack(vs)

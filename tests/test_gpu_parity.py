@@ -21,7 +21,7 @@ import paged_kv_cache_360_b200 as pkv
 from paged_kv_cache_360_b200 import _lib
 from paged_kv_cache_360_b200.workloads import (custom_workload, make_workload, random_block_pairs,
                                                random_slot_mapping, normal_tensor)
-from tests.gpu_helpers import Dev, compare, ensure_built, oracle_decode, words
+from tests.gpu_helpers import Dev, compare, ensure_built, oracle_decode, prefix_rows, words
 
 pytestmark = pytest.mark.gpu
 
@@ -483,18 +483,6 @@ def test_swap_blocks_refuses_pageable_host_memory():
 
 # ------------------------------------------------------------ prefix caching
 
-def _prefix_rows(tokens, Hkv, D, dtype):
-    """K and V rows [len, Hkv, D] where the row at position p depends only on
-    tokens[:p + 1] -- as a model's keys and values do, so that requests with the
-    same prompt prefix have the same rows there."""
-    ks, vs = [], []
-    for p in range(len(tokens)):
-        rng = np.random.default_rng([7] + [int(t) for t in tokens[:p + 1]])
-        ks.append(normal_tensor(rng, (Hkv, D), dtype))
-        vs.append(normal_tensor(rng, (Hkv, D), dtype))
-    return torch.stack(ks), torch.stack(vs)
-
-
 @pytest.mark.parametrize("dtype,D,bs", [(torch.bfloat16, 128, 16), (torch.float16, 64, 32)])
 def test_prefix_cached_requests_share_blocks_and_decode_correctly(dtype, D, bs):
     """Three requests with a common system prompt: the second and third start on
@@ -517,7 +505,7 @@ def test_prefix_cached_requests_share_blocks_and_decode_correctly(dtype, D, bs):
         slots, pairs = pool.reserve_tokens(sid, prompt[n:])
         assert (list(slots), pairs) == model.reserve_tokens(sid, prompt[n:])
         assert pairs == []
-        kr, vr = _prefix_rows(prompt, Hkv, D, dtype)
+        kr, vr = prefix_rows(prompt, Hkv, D, dtype)
         pkv.paged_kv_append(kd, vd, kr[n:].cuda(), vr[n:].cuda(), torch.from_numpy(slots).cuda())
         oracle.append(kw, vw, kr[n:], vr[n:], slots)
         seqs.append(sid)
@@ -544,7 +532,7 @@ def test_prefix_cached_requests_share_blocks_and_decode_correctly(dtype, D, bs):
     code = oracle.BF16 if dtype == torch.bfloat16 else oracle.F16
     ref = np.empty((3, H, D))
     for i, prompt in enumerate(prompts):
-        kr, vr = _prefix_rows(prompt, Hkv, D, dtype)
+        kr, vr = prefix_rows(prompt, Hkv, D, dtype)
         K, V, Q = oracle.widen(words(kr), code), oracle.widen(words(vr), code), \
             oracle.widen(words(q[i]), code)
         for h in range(H):

@@ -18,7 +18,7 @@ import torch
 import oracle
 import paged_kv_cache_360_b200 as pkv
 from paged_kv_cache_360_b200.workloads import custom_workload, normal_tensor
-from tests.gpu_helpers import compare, ensure_built
+from tests.gpu_helpers import compare, ensure_built, prefix_rows, words
 
 pytestmark = pytest.mark.gpu
 
@@ -162,3 +162,51 @@ def test_prefill_llama3_8b_layer_sampled():
         ref = oracle.paged_decode(q[row:row + 1], wl.k_cache, wl.v_cache, wl.block_tables[b:b + 1],
                                   np.array([pos + 1], dtype=np.int32), wl.scale)[0]
         compare(out[row:row + 1], ref[None], what=f"sampled b={b} pos={pos}")
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_prefix_cached_request_prefills_only_its_own_tokens(dtype):
+    """Block manager, prefix cache and chunked prefill together: request B shares
+    request A's system prompt, starts on A's cached full blocks, appends and
+    prefills only its own tokens (a chunk at the end of its context); every
+    query row of both requests matches the oracle's prefill over the whole
+    context, read from the oracle's own copy of the pool."""
+    bs, Hkv, H, D, NB = 16, 2, 8, 128, 64
+    rng = np.random.default_rng(71)
+    system = list(rng.integers(0, 1000, size=70))
+    prompts = [system + list(rng.integers(0, 1000, size=m)) for m in (30, 45)]
+    pool = pkv.Pool(NB, bs, rng.permutation(NB))
+    model = oracle.BlockPoolModel(NB, bs, pool.free_list())
+    k0 = normal_tensor(rng, (NB, Hkv, bs, D), dtype)
+    v0 = normal_tensor(rng, (NB, Hkv, bs, D), dtype)
+    kd, vd = k0.cuda(), v0.cuda()
+    kw, vw = words(k0).copy(), words(v0).copy()
+    scale = float(np.float32(1.0 / np.sqrt(D)))
+    covered_all = []
+    for prompt in prompts:
+        sid, covered = pool.new_cached(prompt)
+        assert (sid, covered) == model.new_cached(prompt)
+        slots, pairs = pool.reserve_tokens(sid, prompt[covered:])
+        assert (list(slots), pairs) == model.reserve_tokens(sid, prompt[covered:])
+        kr, vr = prefix_rows(prompt, Hkv, D, dtype)
+        pkv.paged_kv_append(kd, vd, kr[covered:].cuda(), vr[covered:].cuda(), torch.from_numpy(slots).cuda())
+        oracle.append(kw, vw, kr[covered:], vr[covered:], slots)
+        n = len(prompt) - covered
+        q = normal_tensor(rng, (n, H, D), dtype)
+        table = np.array([pool.table(sid)], dtype=np.int32)
+        lens = np.array([len(prompt)], dtype=np.int32)
+        qs = np.array([0, n], dtype=np.int32)
+        out = torch.zeros((n, H, D), dtype=dtype, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        pkv.paged_attention_prefill(out, q.cuda(), kd, vd, torch.from_numpy(table).cuda(),
+                                    torch.from_numpy(lens).cuda(), torch.from_numpy(qs).cuda(), scale,
+                                    err_flag=err)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        k_or = torch.from_numpy(kw.view(np.int16)).view(dtype).reshape(k0.shape)
+        v_or = torch.from_numpy(vw.view(np.int16)).view(dtype).reshape(v0.shape)
+        compare(out, oracle.paged_prefill(q, k_or, v_or, table, lens, qs, scale),
+                what=f"prefix-cached prefill, {covered} cached tokens")
+        covered_all.append(covered)
+    assert covered_all == [0, 64]              # four full 16-token blocks of the system prompt
+    assert np.array_equal(words(kd.cpu()), kw) and np.array_equal(words(vd.cpu()), vw)
