@@ -199,6 +199,35 @@ def decode_device_sha256() -> str:
     return h.hexdigest()
 
 
+def prefill_device_sha256() -> str:
+    """Hash of the prefill kernel's device code: pkv_prefill.cu up to its host
+    section, and the device headers it includes."""
+    import hashlib
+    csrc = os.path.join(ROOT, "paged_kv_cache_360_b200", "csrc")
+    h = hashlib.sha256()
+    src = open(os.path.join(csrc, "pkv_prefill.cu"), "rb").read()
+    h.update(src[:src.find(b"// ------------------------------------------------------------------ host side")])
+    for name in ("pkv_tc.cuh", "pkv_ptx.cuh"):
+        h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()
+
+
+def read_record(name, sha):
+    """bytes_per_launch from a committed ncu summary profiles/<name> taken on
+    device code with the given hash (else None)."""
+    try:
+        rec = {}
+        for line in open(os.path.join(ROOT, "profiles", name)):
+            if ":" in line and not line.startswith("#"):
+                key, val = line.split(":", 1)
+                rec[key.strip()] = val.strip()
+    except OSError:
+        return None
+    if rec.get("source_sha256") != sha:
+        return None
+    return int(rec["bytes_per_launch"])
+
+
 def traffic_record():
     """DRAM bytes per decode launch from the committed ncu summary
     profiles/decode_traffic.txt, if it was taken on the current decode source
@@ -634,7 +663,8 @@ def run_prefill(args, rank, world, local_rank):
                      "peak_kind": f"{peak_kind} bf16 dense burst",
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "frac_of_sustained": round(achieved / peak_sustained, 4) if peak_sustained else None,
-                     "traffic": None, "algorithmic_flops_per_launch": flops,
+                     "traffic": read_record("prefill_traffic.txt", prefill_device_sha256()),
+                     "algorithmic_flops_per_launch": flops,
                      "avg_launch_ms": round(attn_avg, 5)},
         "e2e": {"value": round(world * flops / (e2e_per_step * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_per_step, 5), "steps": e2e_steps,
