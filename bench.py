@@ -57,6 +57,20 @@ def decode_bytes(lens, wl) -> int:
     return kv + qo + table + 4 * wl.num_seqs
 
 
+def unique_decode_bytes(lens, tables, wl) -> int:
+    """decode_bytes with every physical K/V slot counted once: blocks shared by
+    several sequences (a common prefix) are read from DRAM once, the rest of
+    their reads hit L2."""
+    bs = wl.block_size
+    used = {}
+    for b, L in enumerate(np.asarray(lens, dtype=np.int64)):
+        for i in range(int((L + bs - 1) // bs)):
+            blk = int(tables[b, i])
+            used[blk] = max(used.get(blk, 0), int(min(bs, L - i * bs)))
+    kv = sum(used.values()) * wl.num_kv_heads * wl.head_dim * 2 * 2
+    return decode_bytes(lens, wl) - int(np.sum(lens, dtype=np.int64)) * wl.num_kv_heads * wl.head_dim * 4 + kv
+
+
 def append_bytes(n_tokens, wl) -> int:
     row = wl.num_kv_heads * wl.head_dim * 2
     return n_tokens * (2 * row * 2 + 8)        # read key+value, write them, read the slot
@@ -306,20 +320,33 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
 
-    def timed(graph, steps):
+    spread = {}
+
+    def timed(graph, steps, name=None):
         """Device time (ms) of `steps` back-to-back replays: CUDA events on the
-        launching stream around the whole run, barrier + synchronize on both sides."""
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        launching stream around the whole run, barrier + synchronize on both
+        sides.  Events also split the run into up to 20 equal chunks, whose
+        per-step times give the p10 / median / p90 spread (under `name`)."""
+        chunks = max(1, min(20, steps))
+        marks = [torch.cuda.Event(enable_timing=True) for _ in range(chunks + 1)]
+        bounds = [steps * c // chunks for c in range(chunks + 1)]
         barrier()
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(steps):
-                graph.replay()
-            e1.record(stream)
+            marks[0].record(stream)
+            for c in range(chunks):
+                for _ in range(bounds[c + 1] - bounds[c]):
+                    graph.replay()
+                marks[c + 1].record(stream)
         torch.cuda.synchronize()
         barrier()
-        return e0.elapsed_time(e1)
+        if name:
+            per = sorted(marks[c].elapsed_time(marks[c + 1]) / (bounds[c + 1] - bounds[c])
+                         for c in range(chunks) if bounds[c + 1] > bounds[c])
+            spread[name] = {"p10": round(per[len(per) // 10], 5), "median": round(per[len(per) // 2], 5),
+                            "p90": round(per[(len(per) * 9) // 10 - (1 if len(per) >= 10 else 0)], 5),
+                            "chunks": len(per)}
+        return marks[0].elapsed_time(marks[-1])
 
     sampler = ClockSampler()
     if rank == 0:
@@ -330,9 +357,9 @@ def run_ours(args, rank, world, local_rank):
             g_step.replay()
     torch.cuda.synchronize()
     t_wall0 = time.time()
-    step_ms = timed(g_step, args.steps)          # the timed region: K whole steps
+    step_ms = timed(g_step, args.steps, "step_ms")      # the timed region: K whole steps
     t_wall1 = time.time()
-    decode_ms = timed(g_decode, args.steps)      # the dominant kernels alone, K launches
+    decode_ms = timed(g_decode, args.steps, "decode_ms")  # the dominant kernels alone, K launches
 
     # End to end through the public API: every step copies its inputs from
     # pinned host memory to the device, runs the library's calls and reads the
@@ -441,6 +468,9 @@ def run_ours(args, rank, world, local_rank):
                    "timing": "CUDA events around K back-to-back replays of the step's CUDA graph"},
         "seq_decode_steps_per_s": round(world * B / (ms_per_step * 1e-3), 1),
         "hbm_frac": round(value / world / peak, 4),
+        "hbm_frac_of_nominal_7700": round(value / world / 7700.0, 4),
+        "decode_unique_bytes_gbs": round(unique_decode_bytes(lens, tables, wl) / (decode_avg_ms * 1e-3) / 1e9, 2),
+        "spread_ms_per_step": spread,
         "algorithmic_bytes_per_step": step_bytes,
         "roofline": {"bound": "hbm",
                      "kernel": "paged_attention_decode (balanced decode + chain-merge kernels)"
@@ -468,8 +498,17 @@ def run_ours(args, rank, world, local_rank):
         "clocks": sampler.summary(t_wall0, t_wall1),
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, lens, tables, slots, new_key, new_value,
-                                            budget_s=args.cpu_budget)
+        one = cpu_baseline(wl, lens, tables, slots, new_key, new_value, budget_s=args.cpu_budget)
+        try:
+            allc = cpu_baseline_all_cores(wl, lens, one["sample_seqs"])
+            line["cpu_baseline"] = dict(one, value=allc["value"], cores=allc["cores"],
+                                        seconds=allc["seconds"],
+                                        single_core={"value": one["value"], "seconds": one["seconds"]},
+                                        sample=one["sample"] + f"; timed on {allc['cores']} spawned "
+                                               "processes, one share each, value = sample bytes / "
+                                               "slowest process")
+        except Exception as e:  # the single-core figure stands on its own
+            line["cpu_baseline"] = dict(one, all_cores_error=str(e)[:200])
     return line
 
 
@@ -759,11 +798,64 @@ def cpu_baseline(wl, lens, tables, slots, key, value, budget_s=12.0):
     sub_lens = lens[:n]
     nbytes = sample_bytes(wl, sub_lens, n)
     return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1,
-            "kind": "oracle", "seconds": round(dt, 3),
+            "kind": "oracle", "seconds": round(dt, 3), "sample_seqs": n,
             "seq_decode_steps_per_s": round(n / dt, 3),
             "sample": f"first {n} of {wl.num_seqs} sequences of the {wl.name} batch "
                       f"({int(np.sum(sub_lens))} context tokens): oracle append + decode, 1 pass, "
                       f"single-threaded C float64 on {os.cpu_count()} host cores available"}
+
+
+def _oracle_worker(config, seed, seqs, barrier, results):
+    """Spawned process: rebuild the same batch and step bookkeeping (the
+    generator is a pure function of the seed), wait for the others, then time
+    the oracle on its share of the sample."""
+    import paged_kv_cache_360_b200 as pkv
+    from paged_kv_cache_360_b200.workloads import make_workload
+    import oracle
+    oracle.build()
+    wl = make_workload(config, seed=seed, rank=0)
+    pairs, slots, tables, lens, key, value = build_step(wl, pkv)
+    barrier.wait()
+    t0 = time.perf_counter()
+    _oracle_sample(wl, tables, lens, slots, key, value, seqs)
+    results.put(time.perf_counter() - t0)
+
+
+def cpu_baseline_all_cores(wl, lens, n, max_workers=32):
+    """The same sample as cpu_baseline (the first n sequences), shared out over
+    one spawned process per host core (greedy by length), all starting
+    together; throughput = the sample's bytes / the slowest process's time."""
+    import multiprocessing as mp
+    workers = max(1, min(os.cpu_count() or 1, n, max_workers))
+    shares = [[] for _ in range(workers)]
+    loads = [0] * workers
+    for b in sorted(range(n), key=lambda b: -int(lens[b])):
+        w = loads.index(min(loads))
+        shares[w].append(b)
+        loads[w] += int(lens[b])
+    ctx = mp.get_context("spawn")
+    barrier, results = ctx.Barrier(workers), ctx.Queue()
+    procs = [ctx.Process(target=_oracle_worker, args=(wl.config, wl.seed, sorted(sh), barrier, results))
+             for sh in shares]
+    for pr in procs:
+        pr.start()
+    import queue as _queue
+    times, deadline = [], time.time() + 900
+    try:
+        while len(times) < workers:
+            try:
+                times.append(results.get(timeout=5))
+            except _queue.Empty:
+                if time.time() > deadline or any(pr.exitcode not in (None, 0) for pr in procs):
+                    raise RuntimeError("an oracle process failed or ran past its limit")
+    finally:
+        for pr in procs:
+            pr.join(timeout=30)
+            if pr.is_alive():
+                pr.terminate()
+    dt = max(times)
+    nbytes = sample_bytes(wl, lens[:n], n)
+    return {"value": round(nbytes / dt / 1e9, 4), "cores": workers, "seconds": round(dt, 3)}
 
 
 def run_reference(args, rank, world):
