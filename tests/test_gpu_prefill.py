@@ -210,3 +210,40 @@ def test_prefix_cached_request_prefills_only_its_own_tokens(dtype):
         covered_all.append(covered)
     assert covered_all == [0, 64]              # four full 16-token blocks of the system prompt
     assert np.array_equal(words(kd.cpu()), kw) and np.array_equal(words(vd.cpu()), vw)
+
+
+def _sampled_rows(out, wl, q, qs, lens, nq, rng, count):
+    for _ in range(count):
+        b = int(rng.integers(0, len(lens)))
+        if nq[b] == 0:
+            continue
+        i = int(rng.integers(0, nq[b]))
+        row = int(qs[b]) + i
+        pos = int(lens[b]) - int(nq[b]) + i
+        ref = oracle.paged_decode(q[row:row + 1], wl.k_cache, wl.v_cache, wl.block_tables[b:b + 1],
+                                  np.array([pos + 1], dtype=np.int32), wl.scale)[0]
+        compare(out[row:row + 1], ref[None], what=f"sampled b={b} pos={pos}")
+
+
+def test_prefill_long_context_chunk_sampled():
+    """A 256-token chunk at the end of a 32k-token context (256 kv tiles, the
+    block table fetched in 64 chunks of 32 entries) next to a short prompt."""
+    lens, nq = [32768, 300], [256, 300]
+    wl, q, qs = _case(lens, nq, 32, 8, 128, 16, torch.bfloat16, seed=81)
+    out, err = _run(wl, q, qs)
+    assert err == 0
+    _sampled_rows(out, wl, q, qs, lens, nq, np.random.default_rng(6), 24)
+    # the chunk's last row is the full causal row over all 32768 tokens
+    row = int(qs[1]) - 1
+    ref = oracle.paged_decode(q[row:row + 1], wl.k_cache, wl.v_cache, wl.block_tables[0:1],
+                              np.array([32768], dtype=np.int32), wl.scale)[0]
+    compare(out[row:row + 1], ref[None], what="last row of the 32k context")
+
+
+def test_prefill_multi_head_full_size_sampled():
+    """g = 1 (every query head has its own kv head): 128 query tokens per tile."""
+    lens = [1536, 777, 2048, 40]
+    wl, q, qs = _case(lens, lens, 16, 16, 128, 32, torch.float16, seed=83)
+    out, err = _run(wl, q, qs)
+    assert err == 0
+    _sampled_rows(out, wl, q, qs, lens, lens, np.random.default_rng(7), 24)
