@@ -858,6 +858,56 @@ def cpu_baseline_all_cores(wl, lens, n, max_workers=32):
     return {"value": round(nbytes / dt / 1e9, 4), "cores": workers, "seconds": round(dt, 3)}
 
 
+def run_reference_prefill(args, rank, world):
+    """The oracle as the reference arm of the prefill step: each step is the
+    oracle's append + prefill of the last m query tokens of the first chunked
+    request, m sized so that a step takes about --ref-step-budget seconds."""
+    if rank != 0:
+        return None
+    from paged_kv_cache_360_b200.workloads import make_prefill_workload
+    import oracle
+    import paged_kv_cache_360_b200 as pkv
+    oracle.build()
+    wl = make_prefill_workload(args.prefill_workload, seed=args.seed, rank=0)
+    slots, tables, lens = build_prefill_step(wl, pkv)
+    b = 1 if wl.num_seqs > 1 else 0
+    r0, r1 = int(wl.query_start[b]), int(wl.query_start[b + 1])
+    kw, vw = oracle.words(wl.k_cache), oracle.words(wl.v_cache)
+
+    def step(m):
+        t0 = time.perf_counter()
+        oracle.append(kw, vw, wl.new_key[r1 - m:r1], wl.new_value[r1 - m:r1], slots[r1 - m:r1])
+        oracle.paged_prefill(wl.q[r1 - m:r1], kw, vw, tables[b:b + 1], lens[b:b + 1],
+                             np.array([0, m], dtype=np.int32), wl.scale)
+        return time.perf_counter() - t0
+
+    m = 1
+    dt = step(m)
+    while m < r1 - r0 and dt * 2 < args.ref_step_budget:
+        m = min(r1 - r0, m * 2)
+        dt = step(m)
+    for _ in range(args.warmup):
+        step(m)
+    total = sum(step(m) for _ in range(args.steps))
+    ms = total / args.steps * 1e3
+    fl = prefill_flops([int(lens[b])], [0, m], wl.num_heads, wl.head_dim)
+    tf = fl / (ms * 1e-3) / 1e12
+    sample = (f"each step: oracle append + prefill of the last {m} query tokens of request {b} "
+              f"(context {int(lens[b])}) of the {wl.name} batch, single-threaded C float64")
+    return {"impl": "reference", "metric": PREFILL_METRIC, "value": round(tf, 6), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "query_tokens_sampled": m, "num_heads": wl.num_heads,
+                       "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+                       "block_size": wl.block_size, "seed": args.seed},
+            "cpu_baseline": {"value": round(tf, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(tf, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -934,7 +984,7 @@ def main():
         if world == 1 and args.gpus > 1:
             ap.error("--gpus N > 1 must be launched with torchrun (one process per GPU)")
     if args.impl == "reference":
-        line = run_reference(args, rank, world)
+        line = (run_reference_prefill if args.workload == "prefill" else run_reference)(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
         return
