@@ -25,8 +25,11 @@ append_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
               const int64_t* __restrict__ slot_mapping, int64_t total_chunks,
               int32_t chunks_per_row, int32_t num_kv_heads, int32_t block_size,
               int64_t num_slots, int32_t* err_flag) {
-    // let a decode launched behind this kernel start its set-up now
+    // let a decode launched behind this kernel start its set-up now; this kernel
+    // is itself launched as a programmatic dependent of the previous work in the
+    // stream, so it waits for that work before touching memory
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_chunks;
          i += stride) {
@@ -143,12 +146,22 @@ extern "C" pkv_status paged_kv_append(const pkv_cache_desc* desc, void* k_cache,
     const int64_t total = static_cast<int64_t>(num_tokens) * desc->num_kv_heads * chunks_per_row;
     const int64_t want = (total + kCopyThreads - 1) / kCopyThreads;
     const int grid = static_cast<int>(want < 148 * 16 ? want : 148 * 16);
-    append_kernel<<<grid, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<const uint4*>(key),
-        static_cast<const uint4*>(value), slot_mapping, total, chunks_per_row, desc->num_kv_heads,
-        desc->block_size, static_cast<int64_t>(desc->num_blocks) * desc->block_size, err_flag);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kCopyThreads);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(
+        &cfg, append_kernel, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+        static_cast<const uint4*>(key), static_cast<const uint4*>(value), slot_mapping, total,
+        chunks_per_row, desc->num_kv_heads, desc->block_size,
+        static_cast<int64_t>(desc->num_blocks) * desc->block_size, err_flag);
     note_launches(1);
-    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
     return PKV_OK;
 }

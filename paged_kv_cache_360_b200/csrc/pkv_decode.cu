@@ -273,6 +273,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 //   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
 template <typename T, int D>
 __global__ void __launch_bounds__(D) reduce_kernel(const DecodeArgs a, int32_t max_len) {
+    // a kernel launched behind this one may start its set-up now (it waits for
+    // this grid before touching memory)
+    pdl_launch_dependents();
     pdl_wait_primary();  // the partition kernel's results are visible after this
     const int64_t bh = blockIdx.x;
     const int b = static_cast<int>(bh / a.num_heads);
@@ -804,6 +807,9 @@ __global__ void __launch_bounds__(kReduceThreads) balanced_reduce_kernel(const B
     const int grid = gridDim.x;
     const int group = a.group;
     const int tid = threadIdx.x;
+    // a kernel launched behind this one may start its set-up now (it waits for
+    // this grid before touching memory)
+    pdl_launch_dependents();
 
     // The lengths are an input of the whole step (ready before the decode
     // started), so they are read before waiting for the decode's results.
