@@ -402,6 +402,19 @@ const char* pkv_last_error(void);
 
 const char* pkv_status_string(pkv_status status);
 
+/*
+ * Self-test of the bounded waits (failure detection without a fault): launches
+ * one warp that waits on a shared-memory mbarrier nothing ever arrives on, with
+ * the wait the decode kernels use between their producer and consumers
+ * (which = 0), the decode kernels' abortable wait (which = 1) or the prefill
+ * kernel's wait (which = 2).  The wait gives up by itself -- after about 2^30
+ * SM cycles, half a second at full clock, like every wait in the kernels -- and ORs
+ * PKV_DEVERR_WAIT_TIMEOUT into *err_flag (device int32, required); the context
+ * stays usable.  Stream-ordered; returns PKV_ERR_INVALID_ARG for another `which`
+ * or a null err_flag, PKV_ERR_CUDA if the launch fails.
+ */
+pkv_status pkv_selftest_wait_timeout(int32_t which, int32_t* err_flag, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -22,7 +22,7 @@ __all__ = [
     "paged_kv_append", "copy_blocks", "swap_blocks", "paged_attention_decode",
     "paged_attention_workspace_bytes",
     "paged_attention_decode_static_scratch", "paged_attention_prefill", "Pool",
-    "PkvError", "PoolExhausted", "launch_count", "cache_desc",
+    "PkvError", "PoolExhausted", "launch_count", "selftest_wait_timeout", "cache_desc",
 ]
 
 
@@ -196,6 +196,15 @@ def paged_attention_prefill(out, q, k_cache, v_cache, block_tables, context_lens
 def launch_count() -> int:
     """Kernels libpkv has launched in this process."""
     return int(_lib.load().pkv_launch_count())
+
+
+def selftest_wait_timeout(which, err_flag, stream=None):
+    """Run one bounded wait on an mbarrier nothing arrives on (which = 0: the
+    decode pipeline wait, 1: the decode abortable wait, 2: the prefill wait);
+    it must give up by itself and set DEVERR_WAIT_TIMEOUT in err_flag."""
+    torch = _torch()
+    _lib.check(_lib.load().pkv_selftest_wait_timeout(
+        int(which), _dev(err_flag, "err_flag", torch.int32), _stream(stream)))
 
 
 class Pool:

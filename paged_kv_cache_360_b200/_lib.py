@@ -30,7 +30,7 @@ EXPORTS = (
     "pkv_seq_reserve_tokens", "pkv_seq_new_cached",
     "pkv_seq_cow", "pkv_seq_free", "pkv_seq_swap_out", "pkv_seq_swap_in", "pkv_seq_len", "pkv_seq_block_table", "pkv_pool_block_tables",
     "pkv_pool_refcount", "pkv_pool_free_list", "pkv_pool_stats",
-    "pkv_launch_count", "pkv_last_error", "pkv_status_string",
+    "pkv_launch_count", "pkv_last_error", "pkv_status_string", "pkv_selftest_wait_timeout",
 )
 
 
@@ -105,6 +105,7 @@ def load():
                 "pkv_launch_count": (ctypes.c_uint64, []),
                 "pkv_last_error": (ctypes.c_char_p, []),
                 "pkv_status_string": (ctypes.c_char_p, [st]),
+                "pkv_selftest_wait_timeout": (st, [i32, p, p]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(lib, name)

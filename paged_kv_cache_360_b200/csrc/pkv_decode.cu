@@ -365,15 +365,33 @@ struct BalancedLayout {
     }
 };
 
-// Poll a barrier until the phase with `parity` completes, the limit runs out or
-// another warp has aborted; false unless the phase completed.
+// Poll a barrier until the phase with `parity` completes, about kWaitCycles SM
+// cycles pass or another warp has aborted; false unless the phase completed.
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
                                               const volatile int* abort_word) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    if (mbar_test(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (;;) {
         if (mbar_test(bar, parity)) return true;
-        if ((i & 63) == 63 && *abort_word) return false;
+        if (*abort_word || clock64() - t0 > kWaitCycles) return false;
     }
-    return false;
+}
+
+// Diagnostic (pkv_selftest_wait_timeout): one warp waits on an mbarrier that
+// nothing ever arrives on -- with the plain bounded wait (which = 0) or the
+// abortable one (which = 1) -- and must give up by itself and report it.
+__global__ void selftest_wait_kernel(int which, int32_t* err) {
+    __shared__ __align__(8) uint64_t bar_word;
+    __shared__ int abort_word;
+    const uint32_t bar = smem_addr(&bar_word);
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        abort_word = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const bool ok = which == 0 ? mbar_wait(bar, 0) : wait_or_abort(bar, 0, &abort_word);
+    if (!__all_sync(0xffffffffu, ok) && threadIdx.x == 0) flag(err, PKV_DEVERR_WAIT_TIMEOUT);
 }
 
 // Issue the K and V tiles of one 16-token unit: rows [row0, row0 + 16) of the
@@ -1093,6 +1111,21 @@ size_t balanced_workspace(int grid, int group, int D) {
 }  // namespace pkv
 
 using namespace pkv;
+
+extern "C" pkv_status pkv_selftest_wait_timeout(int32_t which, int32_t* err_flag, void* stream) {
+    if (which < 0 || which > 2) return fail(PKV_ERR_INVALID_ARG, "which must be 0, 1 or 2");
+    if (!err_flag) return fail(PKV_ERR_INVALID_ARG, "err_flag is required");
+    cudaError_t e;
+    if (which == 2) {
+        e = prefill_selftest_wait(err_flag, static_cast<cudaStream_t>(stream));
+    } else {
+        selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(which, err_flag);
+        e = cudaGetLastError();
+    }
+    note_launches(1);
+    if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+    return PKV_OK;
+}
 
 extern "C" size_t paged_attention_workspace_bytes(const pkv_cache_desc* desc, int32_t num_seqs,
                                                   int32_t num_heads, int32_t max_blocks_per_seq,

@@ -155,9 +155,9 @@ __device__ __forceinline__ void flag(int32_t* err, int bit) {
     if (err) atomicOr(err, bit);
 }
 
-// Every wait below gives up after kWaitCycles SM cycles (about half a second):
-// a protocol fault then costs each CTA a bounded delay, never a hang.
-constexpr long long kWaitCycles = 1ll << 30;
+// Every wait below gives up after kWaitCycles SM cycles (about half a second,
+// defined with the other PTX wrappers): a protocol fault then costs each CTA a
+// bounded delay, never a hang.
 
 // Wait that also gives up when another role raised the abort word.
 // Warp-uniform: every lane of the calling warp must call it.
@@ -199,6 +199,22 @@ __device__ __forceinline__ void quiet_wait(uint32_t bar, uint32_t parity) {
     const long long t0 = clock64();
     while (!mbar_test(bar, parity) && clock64() - t0 <= kWaitCycles) {
     }
+}
+
+// Diagnostic (pkv_selftest_wait_timeout, which = 2): one warp waits with the
+// prefill kernel's bounded wait on an mbarrier that nothing ever arrives on; the
+// wait gives up by itself, raises the abort word and reports the timeout.
+__global__ void selftest_wait_kernel(int32_t* err) {
+    __shared__ __align__(8) uint64_t bar_word;
+    __shared__ uint32_t abort_word;
+    const uint32_t bar = smem_addr(&bar_word);
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        abort_word = 0u;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    warp_wait(bar, 0, &abort_word, err);
 }
 
 // Sequence lengths as the kernel uses them: out-of-range values are clamped.
@@ -724,6 +740,13 @@ cudaError_t launch_prefill_dt(int D, int BS, const CUtensorMap& tq, const CUtens
 }
 
 }  // namespace
+}  // namespace pkv
+
+namespace pkv {
+cudaError_t prefill_selftest_wait(int32_t* err, cudaStream_t stream) {
+    selftest_wait_kernel<<<1, 32, 0, stream>>>(err);
+    return cudaGetLastError();
+}
 }  // namespace pkv
 
 using namespace pkv;

@@ -1,8 +1,8 @@
 // pkv_ptx.cuh -- thin inline-PTX wrappers used by the sm_100a kernels.
 //
-// Every wait on an mbarrier is bounded: after kWaitLimit polls it gives up and
-// returns false, and the caller records PKV_DEVERR_WAIT_TIMEOUT and skips the
-// work, so no kernel can spin forever.
+// Every wait on an mbarrier is bounded: after about kWaitCycles SM cycles it
+// gives up and returns false, and the caller records PKV_DEVERR_WAIT_TIMEOUT and
+// skips the work, so no kernel can spin forever.
 #pragma once
 
 #include <cuda.h>
@@ -12,7 +12,11 @@
 
 namespace pkv {
 
-constexpr uint32_t kWaitLimit = 1u << 24;
+// About half a second at the B200's 1.965 GHz SM clock.  The limit is in time,
+// not in polls: a try_wait whose phase has not completed suspends the thread in
+// hardware for microseconds before it returns, so a poll count would give up
+// only after minutes.
+constexpr long long kWaitCycles = 1ll << 30;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -50,9 +54,11 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 
 // Wait until the phase with the given parity has completed; false on timeout.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i)
-        if (mbar_test(bar, parity)) return true;
-    return false;
+    if (mbar_test(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_test(bar, parity))
+        if (clock64() - t0 > kWaitCycles) return false;
+    return true;
 }
 
 // ----------------------------------------------------------------------- TMA

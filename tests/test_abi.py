@@ -107,6 +107,14 @@ def test_status_strings(lib):
         assert lib.pkv_status_string(code).decode() == name
 
 
+def test_selftest_rejects_bad_arguments(lib):
+    # checked on the host before anything is launched
+    assert lib.pkv_selftest_wait_timeout(3, FAKE, None) == 1
+    assert lib.pkv_selftest_wait_timeout(-1, FAKE, None) == 1
+    assert lib.pkv_selftest_wait_timeout(0, None, None) == 1
+    assert "err_flag" in lib.pkv_last_error().decode()
+
+
 def _prefill(lib, desc, **kw):
     a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, tables=FAKE, mb=4, lens=FAKE, qs=FAKE, B=2, T=40,
              H=4, scale=0.1)
