@@ -128,8 +128,11 @@ struct FixedLayout {
     static constexpr int kSmemBytes = kBarOffset + 2 * G::kStages * 8 + 1024;  // + alignment slack
 };
 
+// Three CTAs per SM (at most 128 registers a thread: 15 warps leave 4 per SM
+// sub-partition): a CTA's start-up -- table entries, then the first copies --
+// overlaps the other two CTAs' streaming.
 template <typename T, int D, int BS, bool SPLIT>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 3)
 decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const DecodeArgs a) {
     using G = Geom<D, BS>;
