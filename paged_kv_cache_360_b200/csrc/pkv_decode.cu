@@ -6,8 +6,8 @@
 // What it is: a per-sequence block table maps logical positions to physical
 // blocks.
 //
-// Both schedules below share one CTA shape -- 4 consumer warps + 1 producer warp
-// -- and the tile arithmetic of pkv_attend.cuh:
+// Both schedules below share 4 consumer warps + 1 producer warp (the balanced
+// kernel adds a merge warp) and the tile arithmetic of pkv_attend.cuh:
 //   * the producer issues, per logical block, TMA 2-D tiled loads of the (block,
 //     kv head) K and V tiles -- bs rows x 128 B per 64-column half, 128B swizzle
 //     -- into a ring of shared-memory stages, completion counted on one mbarrier
@@ -272,32 +272,79 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     }
 }
 
-// Merge the partitions of one (sequence, query head) by log-sum-exp, p ascending:
+// Merge the partitions of one (sequence, query head) by log-sum-exp:
 //   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
-template <typename T, int D>
-__global__ void __launch_bounds__(D) reduce_kernel(const DecodeArgs a, int32_t max_len) {
+// With LANES = 1, D threads (one per column) walk p = 0, 1, ... in order.  With
+// many partitions (LANES = 4), LANES groups of D threads split them -- group q
+// takes p = q, q + LANES, ... in ascending order -- so that many partials are
+// read at once, and the groups' sums are added in group order.  Either order
+// depends only on the shapes.
+template <typename T, int D, int LANES>
+__global__ void __launch_bounds__(LANES * D) reduce_kernel(const DecodeArgs a, int32_t max_len) {
     // a kernel launched behind this one may start its set-up now (it waits for
     // this grid before touching memory)
     pdl_launch_dependents();
     pdl_wait_primary();  // the partition kernel's results are visible after this
     const int64_t bh = blockIdx.x;
     const int b = static_cast<int>(bh / a.num_heads);
-    const int d = threadIdx.x;
+    const int tid = threadIdx.x;
     const int L = clamp_len(__ldg(a.context_lens + b), max_len);
     const int n = (L + a.partition_tokens - 1) / a.partition_tokens;
     const float* m = a.ws_m + bh * a.max_partitions;
     const float* l = a.ws_l + bh * a.max_partitions;
     const float* o = a.ws_o + bh * a.max_partitions * D;
-    float M = -INFINITY;
-    for (int p = 0; p < n; ++p) M = fmaxf(M, m[p]);
-    float acc = 0.f, den = 0.f;
-    for (int p = 0; p < n; ++p) {
-        const float f = exp2_approx(m[p] - M);
-        acc += f * o[static_cast<int64_t>(p) * D + d];
-        den += f * l[p];
+    if constexpr (LANES == 1) {
+        const int d = tid;
+        float M = -INFINITY;
+        for (int p = 0; p < n; ++p) M = fmaxf(M, m[p]);
+        float acc = 0.f, den = 0.f;
+        for (int p = 0; p < n; ++p) {
+            const float f = exp2_approx(m[p] - M);
+            acc += f * o[static_cast<int64_t>(p) * D + d];
+            den += f * l[p];
+        }
+        static_cast<T*>(a.out)[bh * D + d] = Pack<T>::one(den > 0.f ? acc / den : 0.f);
+    } else {
+        __shared__ float s_max[LANES * D / 32];
+        __shared__ float s_acc[LANES][D];
+        __shared__ float s_den[LANES];
+        const int q = tid / D;
+        const int d = tid - q * D;
+        // M over all partitions: one strided pass by every thread, then the block
+        float M = -INFINITY;
+        for (int p = tid; p < n; p += LANES * D) M = fmaxf(M, m[p]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        if ((tid & 31) == 0) s_max[tid >> 5] = M;
+        __syncthreads();
+        M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < LANES * D / 32; ++w) M = fmaxf(M, s_max[w]);
+        float acc = 0.f, den = 0.f;
+#pragma unroll 4
+        for (int p = q; p < n; p += LANES) {
+            const float f = exp2_approx(m[p] - M);
+            acc += f * o[static_cast<int64_t>(p) * D + d];
+            den += f * l[p];
+        }
+        s_acc[q][d] = acc;
+        if (d == 0) s_den[q] = den;
+        __syncthreads();
+        if (q == 0) {
+            float sum = s_acc[0][d], dsum = s_den[0];
+#pragma unroll
+            for (int g = 1; g < LANES; ++g) {
+                sum += s_acc[g][d];
+                dsum += s_den[g];
+            }
+            static_cast<T*>(a.out)[bh * D + d] = Pack<T>::one(dsum > 0.f ? sum / dsum : 0.f);
+        }
     }
-    static_cast<T*>(a.out)[bh * D + d] = Pack<T>::one(den > 0.f ? acc / den : 0.f);
 }
+
+// Partitions per (sequence, head) from which the merge splits them over four
+// thread groups.
+constexpr int64_t kWideReduceFrom = 32;
 
 // =========================================================================== balanced
 
@@ -986,7 +1033,8 @@ pkv_status launch_fixed(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
         // in griddepcontrol.wait for the results.
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(num_seqs) * a.num_heads);
-        cfg.blockDim = dim3(D);
+        const bool wide = a.max_partitions >= kWideReduceFrom;
+        cfg.blockDim = dim3((wide ? 4 : 1) * D);
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -994,7 +1042,8 @@ pkv_status launch_fixed(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         const int32_t max_len = a.max_blocks_per_seq * BS;
-        e = cudaLaunchKernelEx(&cfg, reduce_kernel<T, D>, a, max_len);
+        e = wide ? cudaLaunchKernelEx(&cfg, reduce_kernel<T, D, 4>, a, max_len)
+                 : cudaLaunchKernelEx(&cfg, reduce_kernel<T, D, 1>, a, max_len);
         note_launches(1);
         if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
     } else {
