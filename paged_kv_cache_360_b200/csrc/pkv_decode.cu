@@ -866,6 +866,7 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 // Sequences with no tokens get zeros here.
 constexpr int kReduceThreads = 128;
 constexpr int kChainWindow = 32;  // chains up to this many CTAs long are found in one round
+constexpr int kShortChain = 4;    // chains up to this long are merged from registers
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kReduceThreads) balanced_reduce_kernel(const BalancedArgs a) {
@@ -947,21 +948,55 @@ __global__ void __launch_bounds__(kReduceThreads) balanced_reduce_kernel(const B
             const int r = item / (D / 4);
             const int d0 = (item - r * (D / 4)) * 4;
             float M = -INFINITY;
-            for (int k = 0; k < n; ++k) {
-                const int64_t p = static_cast<int64_t>(c + k) * 2 + (k == 0 ? slot : 0);
-                M = fmaxf(M, a.ws_ml[(p * group + r) * 2]);
-            }
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             float den = 0.f;
-            for (int k = 0; k < n; ++k) {
-                const int64_t p = static_cast<int64_t>(c + k) * 2 + (k == 0 ? slot : 0);
-                const float f = exp2_approx(a.ws_ml[(p * group + r) * 2] - M);
-                const float4 o = *reinterpret_cast<const float4*>(a.ws_o + (p * group + r) * D + d0);
-                acc.x += f * o.x;
-                acc.y += f * o.y;
-                acc.z += f * o.z;
-                acc.w += f * o.w;
-                den += f * a.ws_ml[(p * group + r) * 2 + 1];
+            if (n <= kShortChain) {
+                // A short chain's partials are all loaded at once (one round trip
+                // after the decode ends), then combined in the order of the loop
+                // below.
+                float mk[kShortChain], lk[kShortChain];
+                float4 ok[kShortChain];
+#pragma unroll
+                for (int k = 0; k < kShortChain; ++k) {
+                    mk[k] = -INFINITY;
+                    lk[k] = 0.f;
+                    ok[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (k < n) {
+                        const int64_t p = static_cast<int64_t>(c + k) * 2 + (k == 0 ? slot : 0);
+                        mk[k] = a.ws_ml[(p * group + r) * 2];
+                        lk[k] = a.ws_ml[(p * group + r) * 2 + 1];
+                        ok[k] = *reinterpret_cast<const float4*>(a.ws_o + (p * group + r) * D + d0);
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < kShortChain; ++k)
+                    if (k < n) M = fmaxf(M, mk[k]);
+#pragma unroll
+                for (int k = 0; k < kShortChain; ++k) {
+                    if (k < n) {
+                        const float f = exp2_approx(mk[k] - M);
+                        acc.x += f * ok[k].x;
+                        acc.y += f * ok[k].y;
+                        acc.z += f * ok[k].z;
+                        acc.w += f * ok[k].w;
+                        den += f * lk[k];
+                    }
+                }
+            } else {
+                for (int k = 0; k < n; ++k) {
+                    const int64_t p = static_cast<int64_t>(c + k) * 2 + (k == 0 ? slot : 0);
+                    M = fmaxf(M, a.ws_ml[(p * group + r) * 2]);
+                }
+                for (int k = 0; k < n; ++k) {
+                    const int64_t p = static_cast<int64_t>(c + k) * 2 + (k == 0 ? slot : 0);
+                    const float f = exp2_approx(a.ws_ml[(p * group + r) * 2] - M);
+                    const float4 o = *reinterpret_cast<const float4*>(a.ws_o + (p * group + r) * D + d0);
+                    acc.x += f * o.x;
+                    acc.y += f * o.y;
+                    acc.z += f * o.z;
+                    acc.w += f * o.w;
+                    den += f * a.ws_ml[(p * group + r) * 2 + 1];
+                }
             }
             const float inv = den > 0.f ? 1.f / den : 0.f;
             float r0, r1;
