@@ -62,7 +62,7 @@ typedef enum pkv_dtype { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
 #define PKV_DEVERR_BAD_BLOCK_ID 1    /* table entry outside [0, num_blocks): block 0 read instead */
 #define PKV_DEVERR_BAD_CONTEXT_LEN 2 /* context length < 0 or > max_blocks_per_seq*block_size: clamped */
 #define PKV_DEVERR_BAD_SLOT 4        /* slot >= num_blocks*block_size: token skipped */
-#define PKV_DEVERR_WAIT_TIMEOUT 8    /* a pipeline wait ran past its iteration limit: work skipped */
+#define PKV_DEVERR_WAIT_TIMEOUT 8    /* a pipeline wait ran past its time limit (~0.5 s): work skipped */
 #define PKV_DEVERR_BAD_PAIR 16       /* copy pair id outside the pool: pair skipped */
 #define PKV_DEVERR_BAD_QUERY_COUNT 32 /* prefill: query count < 0 or > context length, or a query
                                          row past num_tokens: clamped / not written */
