@@ -116,20 +116,19 @@ def build_step(wl, pkv):
             p = pool.cow(s, last_prefix_block)
             if p:
                 pairs.append(p)
-        for b, s in enumerate(seqs):
-            sl, cp = pool.reserve(s, int(wl.suffix_lens[b]) + 1)
-            pairs.extend(cp)
-            slots.extend(int(x) for x in sl)
+        sl, cp = pool.reserve_batch(seqs, [int(n) + 1 for n in wl.suffix_lens[:len(seqs)]])
+        pairs.extend(cp)
+        slots.extend(int(x) for x in sl)
     else:
         seqs = []
         for b in range(wl.num_seqs):
             s = pool.new_seq()
             pool.reserve(s, int(wl.context_lens[b]) - 1)
             seqs.append(s)
-        for s in seqs:
-            sl, cp = pool.reserve(s, 1)
-            pairs.extend(cp)
-            slots.extend(int(x) for x in sl)
+        # the step's allocation, one call for the whole batch
+        sl, cp = pool.reserve_batch(seqs)
+        pairs.extend(cp)
+        slots.extend(int(x) for x in sl)
     mb = max(len(pool.table(s)) for s in seqs)
     tables, lens = pool.block_tables(seqs, mb, pad=-1)
     pool.close()

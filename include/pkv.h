@@ -314,6 +314,24 @@ pkv_status pkv_seq_reserve(pkv_pool* pool, int32_t seq, int32_t n_tokens, int64_
                            int32_t* cow_pair_out, int32_t* n_cow_out);
 
 /*
+ * One decode step's allocation in one call: for i = 0 .. n_seqs-1, in order,
+ * what pkv_seq_reserve(pool, seqs[i], n_tokens[i], ...) does (n_tokens NULL
+ * means one token each).  slots_out (host int64, sum of the counts) receives the
+ * sequences' slots back to back; copy pairs go to cow_pairs_out (host int32
+ * [cow_cap][2]) in order and *n_cow_out counts them (a sequence needs at most
+ * one, so cow_cap = n_seqs always suffices).  The first sequence that cannot be
+ * served -- free pool exhausted (PKV_ERR_NO_FREE_BLOCK), unknown or swapped out,
+ * or needing a copy past cow_cap (PKV_ERR_INVALID_ARG) -- ends the batch with
+ * that status; the *n_done sequences before it keep their reservations and
+ * their slots and pairs are in the outputs, and nothing of the failing one
+ * changed.  n_cow_out and n_done are required.
+ */
+pkv_status pkv_pool_reserve_batch(pkv_pool* pool, const int32_t* seqs, int32_t n_seqs,
+                                  const int32_t* n_tokens, int64_t* slots_out,
+                                  int32_t* cow_pairs_out, int32_t cow_cap, int32_t* n_cow_out,
+                                  int32_t* n_done);
+
+/*
  * Prefix caching ([glossary], paragraph on prefix caching: requests whose
  * prompts start the same point their block tables at the KV blocks already
  * computed for that start; [ops page] When to use it: a large system prompt

@@ -250,6 +250,35 @@ class Pool:
                                              pair.ctypes.data_as(ctypes.c_void_p), ctypes.byref(n)))
         return slots[:n_tokens], ([(int(pair[0]), int(pair[1]))] if n.value else [])
 
+    def reserve_batch(self, seqs, n_tokens=None):
+        """One decode step's allocation in one call: reserve(seqs[i], n_tokens[i])
+        for every i in order (one token each when n_tokens is None).  Returns
+        (slots int64 array of all sequences back to back, [(src, dst)] copy
+        pairs).  If sequence i cannot be served, raises PoolExhausted or
+        PkvError with .n_done = i and .slots / .pairs of the sequences before
+        it, whose reservations stand."""
+        ids = np.ascontiguousarray(seqs, dtype=np.int32)
+        counts = None if n_tokens is None else np.ascontiguousarray(n_tokens, dtype=np.int32)
+        total = len(ids) if counts is None else int(counts.sum())
+        slots = np.empty(max(1, total), dtype=np.int64)
+        pairs = np.empty((max(1, len(ids)), 2), dtype=np.int32)
+        n_cow, n_done = ctypes.c_int32(), ctypes.c_int32()
+        st = self._lib.pkv_pool_reserve_batch(
+            self._h, ids.ctypes.data_as(ctypes.c_void_p), len(ids),
+            None if counts is None else counts.ctypes.data_as(ctypes.c_void_p),
+            slots.ctypes.data_as(ctypes.c_void_p), pairs.ctypes.data_as(ctypes.c_void_p), len(ids),
+            ctypes.byref(n_cow), ctypes.byref(n_done))
+        served = n_done.value if counts is None else int(counts[:n_done.value].sum())
+        got_slots = slots[:served]
+        got_pairs = [(int(a), int(b)) for a, b in pairs[:n_cow.value]]
+        if st != _lib.PKV_OK:
+            try:
+                _lib.check(st)
+            except _lib.PkvError as e:
+                e.n_done, e.slots, e.pairs = n_done.value, got_slots, got_pairs
+                raise
+        return got_slots, got_pairs
+
     def reserve_tokens(self, seq: int, tokens):
         """reserve() for these token ids, registering the blocks it fills in the
         prefix cache; returns (slots, [(src, dst)] copy pairs)."""

@@ -27,7 +27,7 @@ EXPORTS = (
     "paged_kv_append", "copy_blocks", "swap_blocks", "paged_attention_workspace_bytes", "paged_attention_decode",
     "paged_attention_decode_static_scratch", "paged_attention_prefill",
     "pkv_pool_create", "pkv_pool_destroy", "pkv_seq_new", "pkv_seq_fork", "pkv_seq_reserve",
-    "pkv_seq_reserve_tokens", "pkv_seq_new_cached",
+    "pkv_seq_reserve_tokens", "pkv_seq_new_cached", "pkv_pool_reserve_batch",
     "pkv_seq_cow", "pkv_seq_free", "pkv_seq_swap_out", "pkv_seq_swap_in", "pkv_seq_len", "pkv_seq_block_table", "pkv_pool_block_tables",
     "pkv_pool_refcount", "pkv_pool_free_list", "pkv_pool_stats",
     "pkv_launch_count", "pkv_last_error", "pkv_status_string", "pkv_selftest_wait_timeout",
@@ -92,6 +92,7 @@ def load():
                 "pkv_seq_reserve": (st, [p, i32, i32, p, p, P(i32)]),
                 "pkv_seq_reserve_tokens": (st, [p, i32, p, i32, p, p, P(i32)]),
                 "pkv_seq_new_cached": (st, [p, p, i32, P(i32), P(i32)]),
+                "pkv_pool_reserve_batch": (st, [p, p, i32, p, p, p, i32, P(i32), P(i32)]),
                 "pkv_seq_cow": (st, [p, i32, i32, p, P(i32)]),
                 "pkv_seq_free": (st, [p, i32]),
                 "pkv_seq_swap_out": (st, [p, i32, p, i32, P(i32)]),

@@ -170,6 +170,13 @@ extern "C" pkv_status pkv_seq_fork(pkv_pool* pool, int32_t parent, int32_t* chil
 
 namespace {
 
+// Whether writing n_tokens more tokens to s must first copy its last block: the
+// first token lands in a partly filled block that other sequences share.
+bool needs_copy(const pkv_pool* pool, const pkv_pool::Seq* s, int32_t n_tokens) {
+    const int64_t bs = pool->block_size;
+    return n_tokens > 0 && s->len % bs != 0 && pool->refcount[s->blocks[s->len / bs]] > 1;
+}
+
 pkv_status reserve_impl(pkv_pool* pool, pkv_pool::Seq* s, int32_t n_tokens, int64_t* slots_out,
                         int32_t* cow_pair_out, int32_t* n_cow_out) {
     const int64_t bs = pool->block_size;
@@ -179,8 +186,7 @@ pkv_status reserve_impl(pkv_pool* pool, pkv_pool::Seq* s, int32_t n_tokens, int6
     const int64_t have = (s->len + bs - 1) / bs;
     const int64_t want = (s->len + n_tokens + bs - 1) / bs;
     int64_t need = want - have;
-    const bool cow = n_tokens > 0 && s->len % bs != 0 &&
-                     pool->refcount[s->blocks[s->len / bs]] > 1;
+    const bool cow = needs_copy(pool, s, n_tokens);
     if (cow) {
         need += 1;
         if (!cow_pair_out || !n_cow_out)
@@ -223,6 +229,49 @@ extern "C" pkv_status pkv_seq_reserve(pkv_pool* pool, int32_t seq, int32_t n_tok
         s->tokens.clear();
     }
     return st;
+}
+
+extern "C" pkv_status pkv_pool_reserve_batch(pkv_pool* pool, const int32_t* seqs, int32_t n_seqs,
+                                             const int32_t* n_tokens, int64_t* slots_out,
+                                             int32_t* cow_pairs_out, int32_t cow_cap,
+                                             int32_t* n_cow_out, int32_t* n_done) {
+    if (n_cow_out) *n_cow_out = 0;
+    if (n_done) *n_done = 0;
+    if (!pool || n_seqs < 0 || (n_seqs > 0 && !seqs) || !n_cow_out || !n_done || cow_cap < 0 ||
+        (cow_cap > 0 && !cow_pairs_out))
+        return fail(PKV_ERR_INVALID_ARG, "pkv_pool_reserve_batch: bad argument");
+    int64_t total = 0;
+    for (int32_t i = 0; i < n_seqs; ++i) {
+        const int32_t n = n_tokens ? n_tokens[i] : 1;
+        if (n < 0) return fail(PKV_ERR_INVALID_ARG, "pkv_pool_reserve_batch: negative token count");
+        total += n;
+    }
+    if (total > 0 && !slots_out) return fail(PKV_ERR_INVALID_ARG, "pkv_pool_reserve_batch: slots_out is NULL");
+    // Sequence by sequence, exactly as pkv_seq_reserve; the first failure stops
+    // the batch with the sequences before it served.
+    int64_t off = 0;
+    int32_t ncow = 0;
+    for (int32_t i = 0; i < n_seqs; ++i) {
+        const int32_t n = n_tokens ? n_tokens[i] : 1;
+        pkv_pool::Seq* s = pool->resident(seqs[i]);
+        if (!s)
+            return fail(PKV_ERR_INVALID_ARG, "pkv_pool_reserve_batch: unknown or swapped-out sequence");
+        if (ncow == cow_cap && needs_copy(pool, s, n))
+            return fail(PKV_ERR_INVALID_ARG, "pkv_pool_reserve_batch: more copies than cow_cap");
+        int32_t c = 0;
+        const pkv_status st = reserve_impl(pool, s, n, slots_out + off,
+                                           ncow < cow_cap ? cow_pairs_out + 2 * ncow : nullptr, &c);
+        if (st != PKV_OK) return st;
+        if (n > 0) {  // the token ids are unknown from here on
+            s->tokens_known = false;
+            s->tokens.clear();
+        }
+        off += n;
+        ncow += c;
+        *n_cow_out = ncow;
+        *n_done = i + 1;
+    }
+    return PKV_OK;
 }
 
 extern "C" pkv_status pkv_seq_reserve_tokens(pkv_pool* pool, int32_t seq, const int32_t* tokens,

@@ -202,3 +202,87 @@ def test_library_rejects_misuse():
         pool.free_seq(sid)                       # already freed
     with pytest.raises(PkvError):
         pool.refcount(9)
+
+
+def _same_pools(a, b, live):
+    assert a.free_list() == b.free_list()
+    assert a.stats() == b.stats()
+    for sid in live:
+        assert a.table(sid) == b.table(sid)
+        assert a.length(sid) == b.length(sid)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_batched_reserve_equals_the_sequential_calls(seed):
+    """pkv_pool_reserve_batch against one pkv_seq_reserve per sequence on a twin
+    pool: same slots, copy pairs, tables, free list and statistics, including
+    batches that repeat a sequence, write into shared partly filled blocks, and
+    run the pool dry half way (the served prefix stands)."""
+    rng = np.random.default_rng(1300 + seed)
+    nb, bs = int(rng.integers(16, 96)), int(rng.choice([1, 2, 4, 16]))
+    order = rng.permutation(nb)
+    a, b = Pool(nb, bs, order), Pool(nb, bs, order)
+    live, exhausted = [], 0
+    for _ in range(250):
+        r = rng.random()
+        if r < 0.15 or not live:
+            sa, sb = a.new_seq(), b.new_seq()
+            assert sa == sb
+            live.append(sa)
+        elif r < 0.27:
+            parent = int(live[int(rng.integers(len(live)))])
+            ca, cb = a.fork(parent), b.fork(parent)
+            assert ca == cb
+            live.append(ca)
+        elif r < 0.35 and len(live) > 1:
+            sid = live.pop(int(rng.integers(len(live))))
+            a.free_seq(sid)
+            b.free_seq(sid)
+        else:
+            k = int(rng.integers(1, len(live) + 1))
+            seqs = [int(x) for x in rng.choice(live, size=k, replace=True)]
+            counts = None if rng.random() < 0.5 else [int(x) for x in rng.integers(0, 2 * bs + 2, size=k)]
+            exp_slots, exp_pairs, done, failed = [], [], 0, False
+            for i, sid in enumerate(seqs):
+                try:
+                    s_, p_ = b.reserve(sid, 1 if counts is None else counts[i])
+                except PoolExhausted:
+                    failed = True
+                    break
+                exp_slots += [int(x) for x in s_]
+                exp_pairs += p_
+                done += 1
+            if failed:
+                exhausted += 1
+                with pytest.raises(PoolExhausted) as ei:
+                    a.reserve_batch(seqs, counts)
+                got_s, got_p = ei.value.slots, ei.value.pairs
+                assert ei.value.n_done == done
+            else:
+                got_s, got_p = a.reserve_batch(seqs, counts)
+            assert [int(x) for x in got_s] == exp_slots and got_p == exp_pairs
+        _same_pools(a, b, live)
+    assert exhausted > 0
+
+
+def test_batched_reserve_stops_at_a_copy_past_cow_cap():
+    import ctypes
+    from paged_kv_cache_360_b200 import _lib
+    pool = Pool(8, 4, np.arange(8))
+    s0 = pool.new_seq()
+    pool.reserve(s0, 2)                     # block 0 half full
+    s1 = pool.fork(s0)                      # now shared
+    s2 = pool.new_seq()
+    lib = _lib.load()
+    ids = np.array([s2, s1], dtype=np.int32)
+    slots = np.empty(2, dtype=np.int64)
+    n_cow, n_done = ctypes.c_int32(), ctypes.c_int32()
+    st = lib.pkv_pool_reserve_batch(pool._h, ids.ctypes.data_as(ctypes.c_void_p), 2, None,
+                                    slots.ctypes.data_as(ctypes.c_void_p), None, 0,
+                                    ctypes.byref(n_cow), ctypes.byref(n_done))
+    assert st == 1 and n_done.value == 1 and n_cow.value == 0
+    assert "cow_cap" in lib.pkv_last_error().decode()
+    assert pool.length(s2) == 1 and pool.length(s1) == 2   # s1 untouched
+    # with room for the copy, s1 copies its shared half-full block and goes on
+    got, pairs = pool.reserve_batch([s1])
+    assert len(pairs) == 1 and pairs[0][0] == pool.table(s0)[0] and pool.length(s1) == 3
