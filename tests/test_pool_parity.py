@@ -286,3 +286,33 @@ def test_batched_reserve_stops_at_a_copy_past_cow_cap():
     # with room for the copy, s1 copies its shared half-full block and goes on
     got, pairs = pool.reserve_batch([s1])
     assert len(pairs) == 1 and pairs[0][0] == pool.table(s0)[0] and pool.length(s1) == 3
+
+
+def test_batched_reserve_on_prefix_cached_sequences():
+    """Requests admitted through the prefix cache, then grown by the batched call:
+    same slots, pairs, cache statistics and tables as single calls on a twin pool."""
+    rng = np.random.default_rng(77)
+    nb, bs = 64, 4
+    order = rng.permutation(nb)
+    a, b = Pool(nb, bs, order), Pool(nb, bs, order)
+    stem = [int(x) for x in rng.integers(0, 9, size=10)]
+    live = []
+    for i in range(5):
+        prompt = stem + [int(x) for x in rng.integers(0, 9, size=i)]
+        (sid, covered), rb = a.new_cached(prompt), b.new_cached(prompt)
+        assert (sid, covered) == rb
+        sa, pa = a.reserve_tokens(sid, prompt[covered:])
+        sb, pb = b.reserve_tokens(sid, prompt[covered:])
+        assert list(sa) == list(sb) and pa == pb
+        live.append(sid)
+    assert a.stats()["cached_blocks"] > 0
+    for _ in range(3):
+        counts = [int(x) for x in rng.integers(0, 6, size=len(live))]
+        got_s, got_p = a.reserve_batch(live, counts)
+        exp_s, exp_p = [], []
+        for sid, n in zip(live, counts):
+            s_, p_ = b.reserve(sid, n)
+            exp_s += [int(x) for x in s_]
+            exp_p += p_
+        assert [int(x) for x in got_s] == exp_s and got_p == exp_p
+        _same_pools(a, b, live)
