@@ -98,14 +98,41 @@ def whole_job_gbs(bytes_per_rank_step, world, ms_per_step) -> float:
 
 # ------------------------------------------------------------------ workload
 
-def build_step(wl, pkv):
-    """Host bookkeeping for one decode step with the library's block manager.
+def _reserve_step(pool, seqs, counts):
+    """One step's reservations: the block manager's batched call when it has
+    one, else one reserve per sequence in order (the two agree bit for bit)."""
+    if hasattr(pool, "reserve_batch"):
+        sl, cp = pool.reserve_batch(seqs, counts)
+        return [int(x) for x in sl], [tuple(p) for p in cp]
+    slots, pairs = [], []
+    for i, s in enumerate(seqs):
+        sl, cp = pool.reserve(s, 1 if counts is None else int(counts[i]))
+        slots.extend(int(x) for x in sl)
+        pairs.extend(tuple(p) for p in cp)
+    return slots, pairs
 
+
+def _tables(pool, seqs):
+    mb = max(len(pool.table(s)) for s in seqs)
+    tables = np.full((len(seqs), mb), -1, dtype=np.int32)
+    for i, s in enumerate(seqs):
+        t = pool.table(s)
+        tables[i, :len(t)] = t
+    lens = np.array([pool.length(s) for s in seqs], dtype=np.int32)
+    return tables, lens
+
+
+def build_step(wl, make_pool):
+    """Host bookkeeping for one decode step.
+
+    ``make_pool(num_blocks, block_size, free_order)`` gives the block manager:
+    the library's ``Pool`` on our arm, the oracle's ``BlockPoolModel`` on the
+    reference arm (the two agree bit for bit, tests/test_pool_parity.py).
     Returns (pairs, slots, tables, lens, key, value): the copy pairs, the slots
     of the appended tokens, the block tables and lengths the decode reads, and
     the keys/values appended."""
     bs = wl.block_size
-    pool = pkv.Pool(wl.num_blocks, bs, wl.free_order)
+    pool = make_pool(wl.num_blocks, bs, wl.free_order)
     pairs, slots = [], []
     if wl.prefix_len:
         s0 = pool.new_seq()
@@ -115,10 +142,8 @@ def build_step(wl, pkv):
         for s in seqs:
             p = pool.cow(s, last_prefix_block)
             if p:
-                pairs.append(p)
-        sl, cp = pool.reserve_batch(seqs, [int(n) + 1 for n in wl.suffix_lens[:len(seqs)]])
-        pairs.extend(cp)
-        slots.extend(int(x) for x in sl)
+                pairs.append(tuple(p))
+        sl, cp = _reserve_step(pool, seqs, [int(n) + 1 for n in wl.suffix_lens[:len(seqs)]])
     else:
         seqs = []
         for b in range(wl.num_seqs):
@@ -126,14 +151,23 @@ def build_step(wl, pkv):
             pool.reserve(s, int(wl.context_lens[b]) - 1)
             seqs.append(s)
         # the step's allocation, one call for the whole batch
-        sl, cp = pool.reserve_batch(seqs)
-        pairs.extend(cp)
-        slots.extend(int(x) for x in sl)
-    mb = max(len(pool.table(s)) for s in seqs)
-    tables, lens = pool.block_tables(seqs, mb, pad=-1)
-    pool.close()
+        sl, cp = _reserve_step(pool, seqs, None)
+    pairs.extend(cp)
+    slots.extend(sl)
+    tables, lens = _tables(pool, seqs)
+    if hasattr(pool, "close"):
+        pool.close()
     return (np.array(pairs, dtype=np.int32).reshape(-1, 2), np.array(slots, dtype=np.int64),
             tables, lens, wl.new_key, wl.new_value)
+
+
+def library_pool(pkv):
+    return lambda nb, bs, order: pkv.Pool(nb, bs, order)
+
+
+def oracle_pool():
+    import oracle
+    return lambda nb, bs, order: oracle.BlockPoolModel(nb, bs, order)
 
 
 # ------------------------------------------------------------------- clocks
@@ -268,7 +302,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = make_workload(args.config, seed=args.seed, rank=rank)
-    pairs, slots, tables, lens, new_key, new_value = build_step(wl, pkv)
+    pairs, slots, tables, lens, new_key, new_value = build_step(wl, library_pool(pkv))
 
     k = wl.k_cache.to(dev)
     v = wl.v_cache.to(dev)
@@ -496,6 +530,8 @@ def run_ours(args, rank, world, local_rank):
         "device_err_flag": err_val,
         "clocks": sampler.summary(t_wall0, t_wall1),
     }
+    if world == 1 and not args.no_extras:
+        line.update(extra_records(pkv, dev, peak, args.seed))
     if world == 1 and not args.no_cpu_baseline:
         one = cpu_baseline(wl, lens, tables, slots, new_key, new_value, budget_s=args.cpu_budget)
         try:
@@ -511,16 +547,236 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
+# ------------------------------------------------------------ extra records
+
+def _device_values(shape, dtype, dev, gen):
+    """N(0, 1) values drawn on the device.  The extra records below time
+    kernels whose run time does not depend on the values, so their K/V/q are
+    drawn here instead of by the host generator (which takes minutes for a
+    1 GB pool); shapes, lengths and block tables are the workload's own."""
+    return torch.randn(shape, generator=gen, device=dev, dtype=torch.float32).to(dtype)
+
+
+class _Timer:
+    """Device time of one captured call: CUDA events on its stream."""
+
+    def __init__(self, dev, stream):
+        self.dev, self.stream = dev, stream
+        self.flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # 2x the 126 MB L2
+
+    def capture(self, fn):
+        with torch.cuda.stream(self.stream):
+            fn()                       # eager once (first-call set-up)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            fn()
+        torch.cuda.synchronize()
+        return g
+
+    def back_to_back(self, fn, steps, warmup=5):
+        """Average ms of `steps` replays back to back (inputs larger than L2)."""
+        g = self.capture(fn)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.stream):
+            for _ in range(warmup):
+                g.replay()
+            e0.record(self.stream)
+            for _ in range(steps):
+                g.replay()
+            e1.record(self.stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    def flushed(self, fn, steps, warmup=3):
+        """Average ms of one call with L2 flushed before each (a 256 MB write
+        between calls, outside the events): for inputs that fit in L2."""
+        g = self.capture(fn)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        with torch.cuda.stream(self.stream):
+            for _ in range(warmup):
+                self.flush.zero_()
+                g.replay()
+            for e0, e1 in ev:
+                self.flush.zero_()
+                e0.record(self.stream)
+                g.replay()
+                e1.record(self.stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in ev) / steps
+
+
+def extra_records(pkv, dev, peak, seed):
+    """Kernels of the path beyond the headline workload, each in its own short
+    timed region: the decode on the shared-prefix, long-context and
+    70B-shaped workloads (both schedules where the workload names one), the
+    paged prefill, and the data-movement kernels (append, copy_blocks,
+    swap_blocks)."""
+    from paged_kv_cache_360_b200.workloads import make_workload, make_prefill_workload
+    stream = torch.cuda.Stream(device=dev)
+    timer = _Timer(dev, stream)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234 + int(seed))
+    out = {}
+
+    # ---- decode on the other workloads
+    by_wl = {}
+    for config, P in ((3, 0), (4, 512), (4, 0), (5, 0), (5, 512)):
+        wl = make_workload(config, seed=seed, materialize=False)
+        if config == 3:
+            _, _, tables, lens, _, _ = build_step(wl, library_pool(pkv))
+        else:
+            tables, lens = wl.block_tables, wl.context_lens
+        B, H, D = wl.num_seqs, wl.num_heads, wl.head_dim
+        shape = (wl.num_blocks, wl.num_kv_heads, wl.block_size, D)
+        k = _device_values(shape, wl.dtype, dev, gen)
+        v = _device_values(shape, wl.dtype, dev, gen)
+        q = _device_values((B, H, D), wl.dtype, dev, gen)
+        o = torch.empty_like(q)
+        d_t = torch.from_numpy(np.ascontiguousarray(tables)).to(dev)
+        d_l = torch.from_numpy(np.ascontiguousarray(lens)).to(dev)
+        ws = torch.empty(max(16, pkv.paged_attention_workspace_bytes(k, B, H, d_t.shape[1], P)),
+                         dtype=torch.uint8, device=dev)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+        def decode():
+            pkv.paged_attention_decode(o, q, k, v, d_t, d_l, wl.scale, partition_size=P,
+                                       workspace=ws, err_flag=err)
+
+        nbytes = decode_bytes(lens, wl)
+        fits_l2 = unique_decode_bytes(lens, tables, wl) < 126e6
+        ms = timer.flushed(decode, 100) if fits_l2 else timer.back_to_back(decode, 200)
+        rec = {"workload": wl.name, "schedule": "balanced" if P == 0 else f"fixed partitions of {P}",
+               "num_seqs": B, "ms": round(ms, 5), "algorithmic_bytes": nbytes,
+               "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+               "frac": round(nbytes / (ms * 1e-3) / 1e9 / peak, 4),
+               "seq_decode_steps_per_s": round(B / (ms * 1e-3), 1),
+               "timing": "L2 flushed before each launch, events around it" if fits_l2
+                         else "events around 200 back-to-back decode-only replays",
+               "device_err_flag": int(err.item())}
+        if config == 3:
+            ub = unique_decode_bytes(lens, tables, wl)
+            rec["unique_bytes"] = ub
+            rec["unique_gbs"] = round(ub / (ms * 1e-3) / 1e9, 1)
+            rec["bytes_note"] = ("algorithmic bytes count the shared prefix once per sequence; "
+                                 "unique bytes count every physical slot once")
+        by_wl[f"{config}" if P == wl.partition_size else f"{config}_{'balanced' if P == 0 else f'fixed{P}'}"] = rec
+        del k, v, q, o, ws
+        torch.cuda.empty_cache()
+    out["decode_by_workload"] = by_wl
+
+    # ---- paged prefill
+    pw = make_prefill_workload("prefill-llama3-8b-layer", seed=seed, materialize=False)
+    slots, tables, lens = build_prefill_step(pw, library_pool(pkv))
+    T, H, D = pw.num_tokens, pw.num_heads, pw.head_dim
+    shape = (pw.num_blocks, pw.num_kv_heads, pw.block_size, D)
+    k = _device_values(shape, pw.dtype, dev, gen)
+    v = _device_values(shape, pw.dtype, dev, gen)
+    q = _device_values((T, H, D), pw.dtype, dev, gen)
+    o = torch.empty_like(q)
+    d_t = torch.from_numpy(tables).to(dev)
+    d_l = torch.from_numpy(lens).to(dev)
+    d_qs = torch.from_numpy(pw.query_start).to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def prefill():
+        pkv.paged_attention_prefill(o, q, k, v, d_t, d_l, d_qs, pw.scale, err_flag=err)
+
+    ms = timer.back_to_back(prefill, 50)
+    flops = prefill_flops(lens, pw.query_start, H, D)
+    tpeak, tpeak_sustained, tkind = measured_tensor_peak()
+    tf = flops / (ms * 1e-3) / 1e12
+    out["prefill"] = {"workload": pw.name, "unit": "TFLOP/s", "value": round(tf, 2),
+                      "avg_launch_ms": round(ms, 5), "algorithmic_flops_per_launch": flops,
+                      "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": tpeak,
+                                   "peak_kind": f"{tkind} bf16 dense burst", "frac": round(tf / tpeak, 4),
+                                   "peak_sustained": tpeak_sustained,
+                                   "frac_of_sustained": round(tf / tpeak_sustained, 4)
+                                   if tpeak_sustained else None},
+                      "timing": "events around 50 back-to-back prefill-only replays "
+                                "(the pool is 179 MB, larger than L2)",
+                      "device_err_flag": int(err.item())}
+    del k, v, q, o
+    torch.cuda.empty_cache()
+
+    # ---- data movement: the shared-prefix step's append and copies, a swap
+    wl = make_workload(3, seed=seed, materialize=False)
+    pairs, slots, _, _, _, _ = build_step(wl, library_pool(pkv))
+    shape = (wl.num_blocks, wl.num_kv_heads, wl.block_size, wl.head_dim)
+    k = _device_values(shape, wl.dtype, dev, gen)
+    v = _device_values(shape, wl.dtype, dev, gen)
+    n_new = len(slots)
+    key = _device_values((n_new, wl.num_kv_heads, wl.head_dim), wl.dtype, dev, gen)
+    val = _device_values((n_new, wl.num_kv_heads, wl.head_dim), wl.dtype, dev, gen)
+    d_slots = torch.from_numpy(slots).to(dev)
+    d_pairs = torch.from_numpy(pairs).to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    moves = {}
+    ms = timer.flushed(lambda: pkv.paged_kv_append(k, v, key, val, d_slots, err_flag=err), 100)
+    nb = append_bytes(n_new, wl)
+    moves["append"] = {"what": f"paged_kv_append of the {wl.name} step ({n_new} tokens)",
+                       "ms": round(ms, 5), "bytes": nb, "gbs": round(nb / (ms * 1e-3) / 1e9, 1),
+                       "frac_hbm": round(nb / (ms * 1e-3) / 1e9 / peak, 4)}
+    ms = timer.flushed(lambda: pkv.copy_blocks(k, v, d_pairs, err_flag=err), 100)
+    nb = copy_bytes(len(pairs), wl)
+    moves["copy_blocks"] = {"what": f"copy_blocks of the {wl.name} step ({len(pairs)} pairs)",
+                            "ms": round(ms, 5), "bytes": nb, "gbs": round(nb / (ms * 1e-3) / 1e9, 1),
+                            "frac_hbm": round(nb / (ms * 1e-3) / 1e9 / peak, 4)}
+    # a larger pool of the same geometry (4096 blocks, 128 MiB per K or V pool)
+    # for a 1024-pair copy and a 1024-block swap
+    del k, v
+    rng = np.random.default_rng(seed)
+    shape = (4096,) + shape[1:]
+    k = _device_values(shape, wl.dtype, dev, gen)
+    v = _device_values(shape, wl.dtype, dev, gen)
+    # distinct destinations that are never sources (the pairs a block manager emits)
+    ids = rng.permutation(shape[0])
+    big = np.stack([ids[:1024], ids[1024:2048]], 1).astype(np.int32)
+    d_big = torch.from_numpy(big).to(dev)
+    ms = timer.flushed(lambda: pkv.copy_blocks(k, v, d_big, err_flag=err), 50)
+    nb = copy_bytes(len(big), wl)
+    moves["copy_blocks_1024"] = {"what": "copy_blocks of 1024 random pairs (64 MiB read, 64 MiB "
+                                         "written) in a 4096-block pool of the same geometry",
+                                 "ms": round(ms, 5), "bytes": nb, "gbs": round(nb / (ms * 1e-3) / 1e9, 1),
+                                 "frac_hbm": round(nb / (ms * 1e-3) / 1e9 / peak, 4)}
+    n_swap = 1024
+    blk_bytes = wl.num_kv_heads * wl.block_size * wl.head_dim * 2
+    lst = torch.from_numpy(ids[:n_swap].astype(np.int32)).to(dev)
+    hk = torch.empty((n_swap,) + shape[1:], dtype=wl.dtype).pin_memory()
+    hv = torch.empty((n_swap,) + shape[1:], dtype=wl.dtype).pin_memory()
+    link_bytes = 2 * n_swap * blk_bytes
+    dbuf = torch.empty(link_bytes, dtype=torch.uint8, device=dev)
+    hbuf = torch.empty(link_bytes, dtype=torch.uint8).pin_memory()
+    ms_d2h = timer.flushed(lambda: hbuf.copy_(dbuf, non_blocking=True), 20)
+    ms_h2d = timer.flushed(lambda: dbuf.copy_(hbuf, non_blocking=True), 20)
+    for name, to_host, ref_ms in (("swap_out", True, ms_d2h), ("swap_in", False, ms_h2d)):
+        ms = timer.flushed(lambda: pkv.swap_blocks(k, v, hk, hv, lst, to_host, err_flag=err), 20)
+        link = link_bytes / (ref_ms * 1e-3) / 1e9
+        moves[name] = {"what": f"swap_blocks of {n_swap} blocks "
+                               f"({'device -> pinned host' if to_host else 'pinned host -> device'}, "
+                               f"{link_bytes >> 20} MiB)",
+                       "ms": round(ms, 5), "bytes_over_link": link_bytes,
+                       "gbs": round(link_bytes / (ms * 1e-3) / 1e9, 2),
+                       "link_copy_gbs": round(link, 2),
+                       "frac_of_link_copy": round(link_bytes / (ms * 1e-3) / 1e9 / link, 4),
+                       "link_copy": "one cudaMemcpyAsync of the same bytes, contiguous, pinned"}
+    moves["device_err_flag"] = int(err.item())
+    moves["timing"] = "L2 flushed before each launch, events around it"
+    out["data_movement"] = moves
+    return out
+
+
 # ------------------------------------------------------------------ prefill
 
 PREFILL_METRIC = "paged prefill attention TFLOP/s (causal, % of B200 bf16 dense peak)"
 
 
-def build_prefill_step(wl, pkv):
-    """Block tables, lengths and the query tokens' slots from the library's
-    block manager: every sequence first holds its earlier context, then
-    reserves its query tokens."""
-    pool = pkv.Pool(wl.num_blocks, wl.block_size, wl.free_order)
+def build_prefill_step(wl, make_pool):
+    """Block tables, lengths and the query tokens' slots from a block manager
+    (``make_pool`` as in build_step): every sequence first holds its earlier
+    context, then reserves its query tokens."""
+    pool = make_pool(wl.num_blocks, wl.block_size, wl.free_order)
     seqs = []
     nq = np.diff(wl.query_start)
     for b in range(wl.num_seqs):
@@ -532,9 +788,9 @@ def build_prefill_step(wl, pkv):
         sl, cp = pool.reserve(s, int(nq[b]))
         assert not cp
         slots.extend(int(x) for x in sl)
-    mb = max(len(pool.table(s)) for s in seqs)
-    tables, lens = pool.block_tables(seqs, mb, pad=-1)
-    pool.close()
+    tables, lens = _tables(pool, seqs)
+    if hasattr(pool, "close"):
+        pool.close()
     return np.asarray(slots, dtype=np.int64), tables, lens
 
 
@@ -564,7 +820,7 @@ def run_prefill(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = make_prefill_workload(args.prefill_workload, seed=args.seed, rank=rank)
-    slots, tables, lens = build_prefill_step(wl, pkv)
+    slots, tables, lens = build_prefill_step(wl, library_pool(pkv))
     k, v = wl.k_cache.to(dev), wl.v_cache.to(dev)
     q, key, value = wl.q.to(dev), wl.new_key.to(dev), wl.new_value.to(dev)
     d_slots = torch.from_numpy(slots).to(dev)
@@ -808,12 +1064,11 @@ def _oracle_worker(config, seed, seqs, barrier, results):
     """Spawned process: rebuild the same batch and step bookkeeping (the
     generator is a pure function of the seed), wait for the others, then time
     the oracle on its share of the sample."""
-    import paged_kv_cache_360_b200 as pkv
     from paged_kv_cache_360_b200.workloads import make_workload
     import oracle
     oracle.build()
     wl = make_workload(config, seed=seed, rank=0)
-    pairs, slots, tables, lens, key, value = build_step(wl, pkv)
+    pairs, slots, tables, lens, key, value = build_step(wl, oracle_pool())
     barrier.wait()
     t0 = time.perf_counter()
     _oracle_sample(wl, tables, lens, slots, key, value, seqs)
@@ -865,10 +1120,9 @@ def run_reference_prefill(args, rank, world):
         return None
     from paged_kv_cache_360_b200.workloads import make_prefill_workload
     import oracle
-    import paged_kv_cache_360_b200 as pkv
     oracle.build()
     wl = make_prefill_workload(args.prefill_workload, seed=args.seed, rank=0)
-    slots, tables, lens = build_prefill_step(wl, pkv)
+    slots, tables, lens = build_prefill_step(wl, oracle_pool())
     b = 1 if wl.num_seqs > 1 else 0
     r0, r1 = int(wl.query_start[b]), int(wl.query_start[b + 1])
     kw, vw = oracle.words(wl.k_cache), oracle.words(wl.v_cache)
@@ -912,10 +1166,9 @@ def run_reference(args, rank, world):
         return None
     from paged_kv_cache_360_b200.workloads import make_workload
     import oracle
-    import paged_kv_cache_360_b200 as pkv
     oracle.build()
     wl = make_workload(args.config, seed=args.seed, rank=0)
-    pairs, slots, tables, lens, key, value = build_step(wl, pkv)
+    pairs, slots, tables, lens, key, value = build_step(wl, oracle_pool())
     budget = args.ref_step_budget
     t0 = time.perf_counter()
     _oracle_sample(wl, tables, lens, slots, key, value, [0])
@@ -969,6 +1222,9 @@ def main():
                     help="decode: the decode step (default); prefill: the paged prefill step")
     ap.add_argument("--prefill-workload", default="prefill-llama3-8b-layer")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the extra records (prefill, decode on the other workloads, "
+                         "data-movement kernels) of the decode line")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU time")
     ap.add_argument("--ref-step-budget", type=float, default=3.0,
                     help="seconds of oracle CPU time per reference step")

@@ -158,10 +158,13 @@ size_t paged_attention_workspace_bytes(const pkv_cache_desc* desc, int32_t num_s
  *   t < context_lens[b], K/V of logical token t read from physical block
  *   block_tables[b][t / block_size] at offset t % block_size, kv head
  *   h / (num_heads / num_kv_heads).
- * Arithmetic: fp16/bf16 inputs, fp32 scores, softmax and accumulation, the
- * probabilities rounded to `dtype` for the probability-value product, output
- * rounded to `dtype`.  The reduction order depends only on logical token order,
- * so the result is bit-identical under any permutation of physical blocks.
+ * Arithmetic: fp16/bf16 inputs, fp32 scores, softmax and accumulation.  The
+ * probabilities enter the probability-value product on the tensor cores as a
+ * pair of `dtype` values, p_hi = round(p) and p_lo = round(p - p_hi), each
+ * multiplied by V with fp32 accumulation (two products), so they carry about
+ * 16 significant bits; output rounded to `dtype`.  The reduction order depends
+ * only on logical token order, so the result is bit-identical under any
+ * permutation of physical blocks.
  *   out, q          device [num_seqs][num_heads][head_dim], 16-byte aligned.
  *   k_cache, v_cache device pools, 16-byte aligned (read only).
  *   block_tables    device int32 [num_seqs][max_blocks_per_seq]; entries at or
@@ -242,9 +245,10 @@ pkv_status paged_attention_prefill(const pkv_cache_desc* desc, void* out, const 
  * paged_attention_workspace_bytes(...) exceeds that size are rejected with
  * PKV_ERR_WORKSPACE_TOO_SMALL and nothing is enqueued.  The call allocates
  * nothing.
- *   - The first call on a device looks up the array's device address (once per
- *     device, with that device current); make that first call before any stream
- *     capture.
+ *   - The first call on a device looks up the array's device address with that
+ *     device current, and looks it up again only when the current CUDA context
+ *     is another one than before (after cudaDeviceReset, say); make the first
+ *     call in each context before any stream capture.
  *   - Every call on a device uses the same array, which keeps the last call's
  *     contents; nothing in it needs to start at zero.  Calls that can run at the
  *     same time on the GPU (different streams, no ordering) race on the array

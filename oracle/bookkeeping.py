@@ -309,10 +309,22 @@ class BlockPoolModel:
         }
 
 
-def contiguous_reservation_waste(lengths, reserve_tokens: int) -> dict:
-    """The slab scheme the pages compare against: every request reserves
-    ``reserve_tokens`` contiguous slots up front ("PagedAttention" ops page,
-    Concept -- What it is; KV-cache lesson, problem statement)."""
-    reserved = reserve_tokens * len(lengths)
-    live = sum(min(int(x), reserve_tokens) for x in lengths)
+def contiguous_reservation_waste(lengths, reserve_tokens) -> dict:
+    """The slab scheme the pages compare against: every request reserves a
+    contiguous run of slots up front, sized for the longest output it might
+    produce ("PagedAttention" ops page, Concept -- What it is; KV-cache lesson,
+    problem statement and toy memory map).
+
+    ``reserve_tokens`` is one reservation for every request, or a list with one
+    per request.  A request can hold at most its reservation, so its live slots
+    are min(length, reservation); the rest of the reservation is wasted."""
+    n = len(lengths)
+    if not hasattr(reserve_tokens, "__len__"):
+        reserve = [int(reserve_tokens)] * n
+    else:
+        reserve = [int(r) for r in reserve_tokens]
+        if len(reserve) != n:
+            raise ValueError("one reservation per request")
+    reserved = sum(reserve)
+    live = sum(min(int(x), r) for x, r in zip(lengths, reserve))
     return {"reserved_slots": reserved, "live_slots": live, "wasted_slots": reserved - live}

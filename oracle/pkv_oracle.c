@@ -149,7 +149,9 @@ static int gather_kv(int dtype, const uint16_t* k_cache, const uint16_t* v_cache
  *   tables:   int32 [B][max_blocks];    context_lens: int32 [B]
  *   seqs:     optional list of n_seqs sequence indices to compute (NULL = all B)
  *   out:      double [B][H][D]; only the listed sequences are written.
- * Returns 0, -1 on a bad table entry, -2 on bad shapes, -3 on allocation failure.
+ * Returns 0, -1 on a bad table entry, -2 on bad shapes or a listed index outside
+ * 0 .. B-1 (checked before anything of that sequence is read), -3 on allocation
+ * failure.
  */
 int oracle_paged_decode(int dtype, const uint16_t* q, const uint16_t* k_cache,
                         const uint16_t* v_cache, const int32_t* block_tables,
@@ -167,8 +169,9 @@ int oracle_paged_decode(int dtype, const uint16_t* q, const uint16_t* k_cache,
     int32_t count = seqs ? n_seqs : B;
     for (int32_t i = 0; rc == 0 && i < count; ++i) {
         int32_t b = seqs ? seqs[i] : i;
+        if (b < 0 || b >= B) { rc = -2; break; }
         int64_t L = context_lens[b];
-        if (b < 0 || b >= B || L < 0 || L > max_len) { rc = -2; break; }
+        if (L < 0 || L > max_len) { rc = -2; break; }
         for (int32_t hk = 0; rc == 0 && hk < Hkv; ++hk) {
             if (gather_kv(dtype, k_cache, v_cache, block_tables + (int64_t)b * max_blocks,
                           num_blocks, Hkv, block_size, D, hk, 0, L, K, V) != 0) {

@@ -54,6 +54,10 @@ def _dev(t, name: str, dtype=None):
         return None
     if not t.is_cuda:
         raise PkvError(1, f"{name} must be a CUDA tensor (this library has no CPU path)")
+    cur = _torch().cuda.current_device()
+    if t.device.index != cur:
+        raise PkvError(1, f"{name} is on {t.device} but the current device is cuda:{cur}: "
+                          "the library's calls work on the current device only")
     if not t.is_contiguous():
         raise PkvError(1, f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:

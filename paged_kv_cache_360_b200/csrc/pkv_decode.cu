@@ -1350,23 +1350,69 @@ constexpr size_t kStaticScratchBytes = static_cast<size_t>(PKV_STATIC_SCRATCH_BY
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::atomic<void*> g_scratch_addr[kMaxDevices];
 
-// Device address of g_static_scratch on the current device, looked up once
-// per device.  In host code the array's name is only a stand-in, never a
-// device address, so it must not be passed to a kernel directly.
+// The array's address is a property of the CUDA context that loaded this
+// module: a new context on the same device (after cudaDeviceReset, or a primary
+// context released and retained again) may load it elsewhere.  So the address
+// looked up for a device is kept together with the id of the context it was
+// looked up in (cuCtxGetId: unique for the life of the process), and looked up
+// again when the current context is another one.
+struct ScratchAddress {
+    unsigned long long ctx_id;
+    void* addr;
+};
+std::mutex g_scratch_mu;
+ScratchAddress g_scratch_addr[kMaxDevices];
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Id of the current context, or 0 when there is none yet.
+pkv_status current_context_id(unsigned long long* id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    if (!get_current || !get_id) return fail(PKV_ERR_CUDA, "cuCtxGetCurrent / cuCtxGetId unavailable");
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuCtxGetCurrent failed");
+    *id = 0;
+    if (ctx && get_id(ctx, id) != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuCtxGetId failed");
+    return PKV_OK;
+}
+
+// Device address of g_static_scratch in the current context, looked up once
+// per (device, context) with that device current.  In host code the array's
+// name is only a stand-in, never a device address, so it must not be passed to
+// a kernel directly.
 pkv_status static_scratch_address(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
     if (dev < 0 || dev >= kMaxDevices) return fail(PKV_ERR_UNSUPPORTED, "device index >= 64");
-    void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
-    if (!p) {
-        e = cudaGetSymbolAddress(&p, g_static_scratch);
-        if (e != cudaSuccess || !p)
-            return fail(PKV_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed");
-        g_scratch_addr[dev].store(p, std::memory_order_release);
+    unsigned long long ctx = 0;
+    pkv_status st = current_context_id(&ctx);
+    if (st != PKV_OK) return st;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (ctx != 0 && g_scratch_addr[dev].ctx_id == ctx && g_scratch_addr[dev].addr) {
+        *out = g_scratch_addr[dev].addr;
+        return PKV_OK;
     }
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);  // creates the primary context if needed
+    if (e != cudaSuccess || !p)
+        return fail(PKV_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed");
+    if ((st = current_context_id(&ctx)) != PKV_OK) return st;
+    g_scratch_addr[dev] = ScratchAddress{ctx, p};
     *out = p;
     return PKV_OK;
 }

@@ -40,10 +40,47 @@ class Dev:
         return out
 
 
-def oracle_decode(wl, seqs=None, k=None, v=None, tables=None):
-    return oracle.paged_decode(wl.q, wl.k_cache if k is None else k, wl.v_cache if v is None else v,
-                               wl.block_tables if tables is None else tables, wl.context_lens,
-                               wl.scale, seqs=seqs)
+def oracle_decode(wl, seqs=None, k=None, v=None, tables=None, threads=1):
+    """The oracle's decode of the workload (float64 [B, H, D]).  With
+    threads > 1 the sequences are shared out over that many threads, each
+    calling the oracle on its own sequences (the C oracle runs outside the
+    GIL); every output row is still the oracle's, computed the same way."""
+    k = wl.k_cache if k is None else k
+    v = wl.v_cache if v is None else v
+    tables = wl.block_tables if tables is None else tables
+    if threads <= 1:
+        return oracle.paged_decode(wl.q, k, v, tables, wl.context_lens, wl.scale, seqs=seqs)
+    import concurrent.futures
+    todo = list(range(wl.num_seqs)) if seqs is None else [int(b) for b in seqs]
+    shares = [[] for _ in range(threads)]
+    loads = [0] * threads
+    for b in sorted(todo, key=lambda b: -int(wl.context_lens[b])):
+        i = loads.index(min(loads))
+        shares[i].append(b)
+        loads[i] += int(wl.context_lens[b]) + 1
+    kw, vw = oracle.words(k), oracle.words(v)
+    out = np.zeros((wl.num_seqs, wl.num_heads, wl.head_dim), dtype=np.float64)
+
+    def run(share):
+        part = oracle.paged_decode(wl.q, kw, vw, tables,
+                                   wl.context_lens, wl.scale, seqs=sorted(share))
+        return share, part
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as ex:
+        for share, part in ex.map(run, [s for s in shares if s]):
+            out[share] = part[share]
+    return out
+
+
+PARITY_LOG = []
+
+
+def report_parity(what, mabs, mrel, n):
+    """Record and print one comparison's largest errors (the GPU tests' parity
+    report); with PKV_PARITY_REPORT set, the run's records are also written
+    there as JSON lines at the end of the session."""
+    PARITY_LOG.append({"case": what, "max_abs": mabs, "max_rel": mrel, "elements": n})
+    print(f"parity {what}: max abs {mabs:.3e}, max rel {mrel:.3e} over {n} elements")
 
 
 def compare(gpu_out, ref, seqs=None, what=""):
@@ -59,7 +96,11 @@ def compare(gpu_out, ref, seqs=None, what=""):
             f"{what}: {int(bad.sum())} of {bad.size} elements outside {ATOL} + {RTOL}|ref|; "
             f"max abs {err.max():.3e}, first {idx.tolist()} gpu {g[bad][:5]} ref {ref[bad][:5]}")
     rel = err / np.maximum(np.abs(ref), 1e-30)
-    return float(err.max()), float(np.where(np.abs(ref) > 1e-3, rel, 0).max())
+    mabs = float(err.max()) if err.size else 0.0
+    mrel = float(np.where(np.abs(ref) > 1e-3, rel, 0).max()) if err.size else 0.0
+    if what:
+        report_parity(what, mabs, mrel, int(err.size))
+    return mabs, mrel
 
 
 def words(t):

@@ -32,7 +32,7 @@ def test_decode_bytes_by_enumeration():
 
 def test_unique_bytes_count_shared_blocks_once():
     wl = make_workload(3, seed=0, materialize=False)
-    _, _, tables, lens, _, _ = bench.build_step(wl, pkv)
+    _, _, tables, lens, _, _ = bench.build_step(wl, bench.library_pool(pkv))
     logical, unique = bench.decode_bytes(lens, wl), bench.unique_decode_bytes(lens, tables, wl)
     per_token = wl.num_kv_heads * wl.head_dim * 4
     slots = set()
@@ -42,14 +42,14 @@ def test_unique_bytes_count_shared_blocks_once():
     assert logical - unique == (int(lens.sum()) - len(slots)) * per_token
     assert unique < logical
     wl2 = make_workload(2, seed=0, materialize=False)
-    _, _, t2, l2, _, _ = bench.build_step(wl2, pkv)
+    _, _, t2, l2, _, _ = bench.build_step(wl2, bench.library_pool(pkv))
     assert bench.unique_decode_bytes(l2, t2, wl2) == bench.decode_bytes(l2, wl2)   # no sharing
 
 
 @pytest.mark.parametrize("name", ["prefill-tiny", "prefill-llama3-8b-layer"])
 def test_prefill_step_matches_the_model(name):
     wl = make_prefill_workload(name, seed=2, materialize=False)
-    slots, tables, lens = bench.build_prefill_step(wl, pkv)
+    slots, tables, lens = bench.build_prefill_step(wl, bench.library_pool(pkv))
     model = BlockPoolModel(wl.num_blocks, wl.block_size, wl.free_order)
     nq = np.diff(wl.query_start)
     seqs = [model.new_seq() for _ in range(wl.num_seqs)]
@@ -66,3 +66,23 @@ def test_prefill_step_matches_the_model(name):
         assert list(tables[b, :len(t)]) == t and all(x == -1 for x in tables[b, len(t):])
     assert list(lens) == list(wl.context_lens)
     assert int(wl.query_start[-1]) == len(slots)
+
+
+@pytest.mark.parametrize("config", [1, 2, 3, 5])
+def test_both_arms_build_the_same_step(config):
+    """The reference arm builds the step with the oracle's block-manager model,
+    our arm with the library's: pairs, slots, tables and lengths agree exactly."""
+    wl = make_workload(config, seed=1, materialize=False)
+    ours = bench.build_step(wl, bench.library_pool(pkv))
+    ref = bench.build_step(wl, bench.oracle_pool())
+    for a, b in zip(ours[:4], ref[:4]):
+        assert a.dtype == b.dtype and np.array_equal(a, b)
+    assert np.array_equal(ours[3], wl.context_lens)
+
+
+def test_both_arms_build_the_same_prefill_step():
+    wl = make_prefill_workload("prefill-llama3-8b-layer", seed=1, materialize=False)
+    ours = bench.build_prefill_step(wl, bench.library_pool(pkv))
+    ref = bench.build_prefill_step(wl, bench.oracle_pool())
+    for a, b in zip(ours, ref):
+        assert a.dtype == b.dtype and np.array_equal(a, b)

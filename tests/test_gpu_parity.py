@@ -11,6 +11,7 @@ permutation and copy-on-write must leave the output bit-identical.
 
 import ctypes
 import math
+import os
 
 import numpy as np
 import pytest
@@ -119,7 +120,7 @@ def test_decode_ragged_all_partitions(dtype, D, bs, group):
     ref = oracle_decode(wl)
     for P in (0, bs, 64, 96 if bs == 16 else 128, 512, 1 << 20):
         out = dev.decode(partition_size=P)
-        compare(out, ref, what=f"P={P}")
+        compare(out, ref, what=f"ragged {str(dtype)[6:]} D={D} bs={bs} g={group} P={P}")
         assert dev.err.item() == 0
 
 
@@ -130,7 +131,7 @@ def test_decode_group_of_sixteen(dtype):
     dev = Dev(wl)
     ref = oracle_decode(wl)
     for P in (0, 128):
-        compare(dev.decode(P), ref, what=f"g=16 P={P}")
+        compare(dev.decode(P), ref, what=f"g=16 {str(dtype)[6:]} P={P}")
 
 
 @pytest.mark.parametrize("dtype", DTYPES)
@@ -186,7 +187,7 @@ def test_decode_ignores_garbage_past_the_last_token(dtype):
     for P in (0, 32):
         out = dev.decode(P)
         assert torch.isfinite(out).all()
-        compare(out, ref, what=f"garbage tail P={P}")
+        compare(out, ref, what=f"garbage tail {str(dtype)[6:]} P={P}")
 
 
 def test_decode_flags_bad_table_entries_and_lengths():
@@ -219,24 +220,22 @@ def test_decode_rejects_host_tensors_and_small_workspace():
 
 # ---------------------------------------------------------- full-size workloads
 
-def _sample(wl, n):
-    """The longest, the shortest and a seeded spread of sequences."""
-    order = np.argsort(wl.context_lens)
-    pick = set([int(order[0]), int(order[-1])])
-    pick.update(np.random.default_rng(0).choice(wl.num_seqs, size=min(n, wl.num_seqs), replace=False).tolist())
-    return sorted(pick)
+ORACLE_THREADS = max(1, min(16, os.cpu_count() or 1))
 
 
 @pytest.mark.parametrize("config", [1, 2, 4, 5])
 def test_full_size_workload(config):
+    """Every output element of the full-size workload against the oracle, with
+    the partition size the bench uses (0 = the balanced schedule; the
+    long-context workload's fixed 512-token partitions)."""
     wl = make_workload(config, seed=0)
     dev = Dev(wl)
-    P = wl.partition_size  # 0 = the library's choice, as the bench runs it
+    P = wl.partition_size
     out = dev.decode(P)
     assert dev.err.item() == 0
-    seqs = None if config in (1, 2) else _sample(wl, 24)
-    ref = oracle_decode(wl, seqs=seqs)
-    mabs, mrel = compare(out, ref, seqs=seqs, what=f"config {config}")
+    ref = oracle_decode(wl, threads=ORACLE_THREADS)
+    mabs, mrel = compare(out, ref, what=f"config {config} ({wl.name}), "
+                                         f"{'balanced' if P == 0 else f'fixed P={P}'}")
     assert math.isfinite(mabs)
 
 
@@ -352,7 +351,7 @@ def test_balanced_many_short_and_empty_sequences(dtype, D, bs, group):
     dev = Dev(wl)
     out = dev.decode(0)
     assert dev.err.item() == 0
-    compare(out, oracle_decode(wl), what="balanced short")
+    compare(out, oracle_decode(wl), what=f"balanced 700 short {str(dtype)[6:]} D={D} bs={bs} g={group}")
     assert torch.all(out[torch.from_numpy(lens == 0)] == 0)
 
 
@@ -387,13 +386,17 @@ def test_balanced_large_batch():
     compare(out, oracle_decode(wl), what="balanced large batch")
 
 
-def test_balanced_full_size_long_context():
-    wl = make_workload(4, seed=0)
+@pytest.mark.parametrize("config,P", [(4, 0), (5, 512), (2, 512)])
+def test_full_size_other_schedule(config, P):
+    """The full-size workloads on the schedule the bench does not use by
+    default (balanced for the long-context workload, fixed 512-token
+    partitions for the others), every output element against the oracle."""
+    wl = make_workload(config, seed=0)
     dev = Dev(wl)
-    out = dev.decode(0)
+    out = dev.decode(P)
     assert dev.err.item() == 0
-    seqs = _sample(wl, 3)
-    compare(out, oracle_decode(wl, seqs=seqs), seqs=seqs, what="config 4 balanced")
+    compare(out, oracle_decode(wl, threads=ORACLE_THREADS),
+            what=f"config {config} ({wl.name}), {'balanced' if P == 0 else f'fixed P={P}'}")
 
 
 # ------------------------------------------------------------ swap (preemption)

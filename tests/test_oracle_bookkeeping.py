@@ -284,6 +284,37 @@ def test_toy_memory_map_illustration():
     assert pool.stats()["free_blocks"] == int(spec["paged_free"][0][0])
 
 
+def check_contiguous_reservation_waste(fn):
+    """Exact pins of the slab scheme's accounting (``fn`` is the function under
+    test, so that the mutation tests can hand in broken copies):
+
+    * the lesson's toy memory map (tests/golden/toy_memory_map.txt): twelve
+      slots of four tokens; A holds 14 tokens in a reservation of 6 slots, B 9
+      tokens in 5 slots, so the contiguous row leaves exactly 1 slot free;
+    * a batch worked by hand with one request longer than its reservation (a
+      slab holds at most what was reserved): lengths 5, 12, 3, 0 with 8 tokens
+      reserved each give 32 reserved, 5 + 8 + 3 + 0 = 16 live, 16 wasted;
+    * an empty batch reserves nothing.
+    """
+    spec = {}
+    for raw in open(f"{GOLDEN}/toy_memory_map.txt"):
+        line = raw.split("#", 1)[0].split()
+        if line:
+            spec.setdefault(line[0], []).append(line[1:])
+    slots, bs = int(spec["slots"][0][0]), int(spec["block_size"][0][0])
+    lengths = [int(r[1]) for r in spec["request"]]
+    reserve = [int(r[3]) * bs for r in spec["request"]]
+    toy = fn(lengths, reserve)
+    assert toy == {"reserved_slots": 44, "live_slots": 23, "wasted_slots": 21}
+    assert (slots * bs - toy["reserved_slots"]) // bs == int(spec["contiguous_free"][0][0]) == 1
+    assert fn([5, 12, 3, 0], 8) == {"reserved_slots": 32, "live_slots": 16, "wasted_slots": 16}
+    assert fn([], 8) == {"reserved_slots": 0, "live_slots": 0, "wasted_slots": 0}
+
+
+def test_contiguous_reservation_waste_exact():
+    check_contiguous_reservation_waste(contiguous_reservation_waste)
+
+
 def test_fragmentation_context_on_synthetic_lengths():
     """Context only (not a pin): paged waste vs a max-length slab per request on
     the long-context mixes; the glossary page quotes <4 % vs 60-80 %."""

@@ -1,6 +1,7 @@
 """The oracle's pins must reject plausible mistakes (no GPU).
 
-Each mutant below is a copy of oracle/pkv_oracle.c with one deliberate
+Each mutant below is a copy of oracle/pkv_oracle.c (or, for WASTE_MUTANTS, of
+the bookkeeping model's slab-waste function) with one deliberate
 mistake -- a wrong index, a dropped term, a wrong sign, a transposed operand, a
 wrong constant.  It is compiled on the CPU and test_oracle_pins.py is run
 against it in a child process (PKV_ORACLE_LIB points the oracle at the
@@ -61,6 +62,20 @@ MUTANTS = {
     "prefill GQA mapping interleaved": ("int32_t h = hk * group + j;", "int32_t h = hk + j * Hkv;"),
     "swap direction inverted": ("        if (to_host) {\n            memcpy(hk, pk,",
                                 "        if (!to_host) {\n            memcpy(hk, pk,"),
+    "listed sequence index not checked": ("        if (b < 0 || b >= B) { rc = -2; break; }\n", ""),
+}
+
+# Mutants of the bookkeeping model's slab-waste accounting (Python): each is
+# the function's source with one mistake, run against the exact pins of
+# test_oracle_bookkeeping.check_contiguous_reservation_waste.
+WASTE_MUTANTS = {
+    "live not clamped to the reservation": ("min(int(x), r)", "int(x)"),
+    "live clamped the wrong way": ("min(int(x), r)", "max(int(x), r)"),
+    "reserved counts one request too few": ("reserved = sum(reserve)", "reserved = sum(reserve[1:])"),
+    "reserved off by one slot": ("reserved = sum(reserve)", "reserved = sum(reserve) + 1"),
+    "wasted reversed": ('"wasted_slots": reserved - live', '"wasted_slots": live - reserved'),
+    "one reservation for all, the first": ("reserve = [int(r) for r in reserve_tokens]",
+                                           "reserve = [int(reserve_tokens[0])] * n"),
 }
 
 
@@ -86,6 +101,30 @@ def test_every_mutant_is_caught():
         with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 2)) as ex:
             results = list(ex.map(lambda kv: _run_mutant(kv[0], *kv[1], tmp), MUTANTS.items()))
     survivors = [name for name, rc in results if rc == 0]
+    assert not survivors, f"pins did not catch: {survivors}"
+
+
+def _waste_variant(old, new):
+    import inspect
+    import textwrap
+    from oracle import bookkeeping
+    src = textwrap.dedent(inspect.getsource(bookkeeping.contiguous_reservation_waste))
+    assert src.count(old) == 1, old
+    ns = {}
+    exec(src.replace(old, new), ns)
+    return ns["contiguous_reservation_waste"]
+
+
+def test_every_waste_mutant_is_caught():
+    from tests.test_oracle_bookkeeping import check_contiguous_reservation_waste
+    check_contiguous_reservation_waste(_waste_variant("reserved = ", "reserved = "))
+    survivors = []
+    for name, (old, new) in WASTE_MUTANTS.items():
+        try:
+            check_contiguous_reservation_waste(_waste_variant(old, new))
+        except AssertionError:
+            continue
+        survivors.append(name)
     assert not survivors, f"pins did not catch: {survivors}"
 
 

@@ -171,6 +171,35 @@ def test_sequence_subset_matches_full():
     assert np.array_equal(part[1], full[1]) and np.all(part[0] == 0)
 
 
+def test_sequence_index_outside_the_batch_is_rejected():
+    """A listed sequence index outside 0 .. B-1 returns -2 before anything of
+    that sequence is read.  The call goes straight to the C function with one
+    spare (valid) length and one spare output row behind the batch, so an
+    oracle that skipped the check would compute that row and return 0 instead
+    of faulting."""
+    import ctypes
+    q, k, v, tables, lens, MB = _identity_case(seed=32, lens=(13, 29))
+    B, H, D = q.shape
+    NB, Hkv, bs, _ = k.shape
+    lens_spare = np.array(list(lens) + [5], dtype=np.int32)
+    tables_spare = np.concatenate([tables, tables[:1]]).astype(np.int32)
+    q_spare = np.ascontiguousarray(np.concatenate([oracle.words(q), oracle.words(q)[:1]]))
+    kw, vw = oracle.words(k), oracle.words(v)
+    out = np.zeros((B + 1, H, D), dtype=np.float64)
+    ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    for bad in (B, -1):
+        sel = np.array([0, bad], dtype=np.int32)
+        out[:] = 0
+        rc = oracle._load().oracle_paged_decode(
+            oracle.BF16, ptr(q_spare[1:] if bad < 0 else q_spare), ptr(kw), ptr(vw),
+            ptr(tables_spare[1:] if bad < 0 else tables_spare), MB,
+            ptr(lens_spare[1:] if bad < 0 else lens_spare), B, H, Hkv, D, bs, NB, 0.3, ptr(sel),
+            len(sel), ptr(out[1:] if bad < 0 else out))
+        assert rc == -2, (bad, rc)
+    with pytest.raises(ValueError):
+        oracle.paged_decode(q, k, v, tables, lens, 0.3, seqs=[0, B])
+
+
 def _kv_rows(words, Hkv, D):
     """Pool [NB, Hkv, bs, D] as [Hkv, NB*bs, D]: row s is slot s (a reshape)."""
     NB, _, bs, _ = words.shape
