@@ -647,6 +647,32 @@ def extra_records(pkv, dev, peak, seed):
         nbytes = decode_bytes(lens, wl)
         fits_l2 = unique_decode_bytes(lens, tables, wl) < 126e6
         ms = timer.flushed(decode, 100) if fits_l2 else timer.back_to_back(decode, 200)
+        if config == 3:
+            # the same batch through the shared-prefix decode: the groups come
+            # from the tables (every sequence shares the prompt's full blocks)
+            gs, gb = pkv.shared_prefix_groups(tables, lens, wl.block_size)
+            ws_sp = torch.empty(max(256, pkv.paged_attention_shared_prefix_workspace_bytes(
+                k, B, H, d_t.shape[1], gs, gb)), dtype=torch.uint8, device=dev)
+            o_sp = torch.empty_like(q)
+
+            def decode_sp():
+                pkv.paged_attention_decode_shared_prefix(o_sp, q, k, v, d_t, d_l, wl.scale, gs, gb,
+                                                         workspace=ws_sp, err_flag=err)
+
+            ms_sp = timer.flushed(decode_sp, 100)
+            ub = unique_decode_bytes(lens, tables, wl)
+            by_wl["3_shared_prefix"] = {
+                "workload": wl.name, "schedule": "shared-prefix decode (prefix tiles on tcgen05 + "
+                                                 "balanced decode of each sequence's own tokens)",
+                "groups": {"group_start": [int(x) for x in gs], "shared_blocks": [int(x) for x in gb]},
+                "num_seqs": B, "ms": round(ms_sp, 5), "algorithmic_bytes": nbytes,
+                "gbs": round(nbytes / (ms_sp * 1e-3) / 1e9, 1),
+                "frac": round(nbytes / (ms_sp * 1e-3) / 1e9 / peak, 4),
+                "unique_bytes": ub, "unique_gbs": round(ub / (ms_sp * 1e-3) / 1e9, 1),
+                "unique_frac": round(ub / (ms_sp * 1e-3) / 1e9 / peak, 4),
+                "speedup_vs_balanced": round(ms / ms_sp, 3),
+                "seq_decode_steps_per_s": round(B / (ms_sp * 1e-3), 1),
+                "timing": "L2 flushed before each launch, events around it"}
         rec = {"workload": wl.name, "schedule": "balanced" if P == 0 else f"fixed partitions of {P}",
                "num_seqs": B, "ms": round(ms, 5), "algorithmic_bytes": nbytes,
                "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),

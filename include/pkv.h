@@ -193,6 +193,71 @@ pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* out, const v
                                   void* stream);
 
 /*
+ * Decode attention for a batch in which groups of sequences share the first
+ * blocks of their block tables -- a common prompt prefix whose blocks every
+ * sharing table points at ([ops page] At a glance: shared prompt blocks are
+ * referenced by every table that uses them; How it works: sharing with
+ * reference counts and copy on write; [glossary] prefix caching).  The result
+ * is paged_attention_decode's (same definition, same precision rules); only
+ * the schedule differs:
+ *   - the decode queries of 128 / g sequences of a group times the g heads of
+ *     one kv head form one 128-row tile that attends to the group's shared
+ *     blocks on the tensor cores (tcgen05), so each shared K/V row is read once
+ *     per tile instead of once per sequence; chunks of 128 or 256 shared tokens
+ *     leave un-normalised partials (m, l, O) in the workspace;
+ *   - the balanced decode attends every sequence to its own tokens (those past
+ *     the shared ones) and folds the prefix partials of its rows into its
+ *     log-sum-exp merge, in a fixed order (warps, then prefix chunks).
+ * The reduction order depends only on the shapes and the groups, so results
+ * are bit-identical under any permutation of physical blocks; they differ from
+ * paged_attention_decode's by rounding only.
+ *   group_start          HOST int32 [num_groups + 1]: group i is sequences
+ *                        group_start[i] .. group_start[i+1] - 1 (strictly
+ *                        increasing, group_start[num_groups] <= num_seqs);
+ *                        sequences outside every group are decoded as usual.
+ *   group_shared_blocks  HOST int32 [num_groups]: the first
+ *                        group_shared_blocks[i] entries of every table row of
+ *                        group i are the same physical blocks, all full
+ *                        (0 = nothing shared).  They are read from the row of
+ *                        the group's first sequence; each sequence's
+ *                        context_len must be at least group_shared_blocks[i] *
+ *                        block_size (else PKV_DEVERR_BAD_CONTEXT_LEN and that
+ *                        output is undefined).
+ *   num_groups           0 .. 64.
+ *   num_heads / num_kv_heads must be a power of two <= 16 when a group shares
+ *   blocks (PKV_ERR_UNSUPPORTED otherwise).
+ *   workspace            device, >= paged_attention_shared_prefix_workspace_bytes
+ *                        (...) for the same arguments, 256-byte aligned.
+ * Other arguments, layouts and errors as paged_attention_decode (the schedule
+ * is always the balanced one).  The host arrays are read during the call only.
+ */
+pkv_status paged_attention_decode_shared_prefix(const pkv_cache_desc* desc, void* out,
+                                                const void* q, const void* k_cache,
+                                                const void* v_cache, const int32_t* block_tables,
+                                                int32_t max_blocks_per_seq,
+                                                const int32_t* context_lens, int32_t num_seqs,
+                                                int32_t num_heads, float scale,
+                                                const int32_t* group_start,
+                                                const int32_t* group_shared_blocks,
+                                                int32_t num_groups, void* workspace,
+                                                size_t workspace_bytes, int32_t* err_flag,
+                                                void* stream);
+
+/*
+ * Workspace bytes of paged_attention_decode_shared_prefix: the balanced
+ * decode's workspace (paged_attention_workspace_bytes with partition_size 0)
+ * rounded up to 256 bytes, then float partial outputs [S][head_dim] and
+ * (m, l) pairs [S][2], S = sum over groups that share blocks of (sequences x
+ * num_heads x chunks), chunks = ceil(shared tokens / (128 x tiles per chunk)),
+ * 1 or 2 tiles per chunk.  0 on invalid arguments.
+ */
+size_t paged_attention_shared_prefix_workspace_bytes(const pkv_cache_desc* desc, int32_t num_seqs,
+                                                     int32_t num_heads, int32_t max_blocks_per_seq,
+                                                     const int32_t* group_start,
+                                                     const int32_t* group_shared_blocks,
+                                                     int32_t num_groups);
+
+/*
  * Paged prefill attention: the prompt phase through the same block table
  * ([ops page] How it works: attention reads keys and values through the block
  * table; Concept: processing the prompt is the compute-bound phase, generation
@@ -413,6 +478,29 @@ pkv_status pkv_pool_refcount(const pkv_pool* pool, int32_t block, int32_t* refco
 pkv_status pkv_pool_free_list(const pkv_pool* pool, int32_t* out, int32_t cap, int32_t* n);
 
 pkv_status pkv_pool_stats(const pkv_pool* pool, pkv_stats* stats);
+
+/*
+ * Shared-prefix groups of a batch for paged_attention_decode_shared_prefix,
+ * from host copies of its block tables (int32 [num_seqs][max_blocks_per_seq])
+ * and lengths (int32 [num_seqs]).  Sequences that point their tables at the
+ * same leading blocks share those blocks' keys and values ([ops page] At a
+ * glance and How it works: forked sequences share blocks by reference).
+ * Walking the batch in order, a group starts at sequence i and takes i + 1,
+ * i + 2, ... while the number of leading entries they all have in common with
+ * row i -- counting only blocks that are full in every sequence taken -- stays
+ * >= min_shared_blocks; it is kept if it holds >= min_group_seqs sequences,
+ * else the walk moves on to i + 1.  A gap between two kept groups is written
+ * as a group that shares nothing (group_start must be back to back).  Outputs:
+ * group_start [max_groups + 1], group_shared_blocks [max_groups], *num_groups
+ * <= max_groups (groups that do not fit are dropped: their sequences are then
+ * decoded as usual).  Host memory only; deterministic.
+ */
+pkv_status pkv_shared_prefix_groups(const int32_t* block_tables, int32_t num_seqs,
+                                    int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                    int32_t block_size, int32_t min_group_seqs,
+                                    int32_t min_shared_blocks, int32_t max_groups,
+                                    int32_t* group_start, int32_t* group_shared_blocks,
+                                    int32_t* num_groups);
 
 /* --------------------------------------------------------------- diagnostics */
 

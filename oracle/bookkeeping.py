@@ -328,3 +328,58 @@ def contiguous_reservation_waste(lengths, reserve_tokens) -> dict:
     reserved = sum(reserve)
     live = sum(min(int(x), r) for x, r in zip(lengths, reserve))
     return {"reserved_slots": reserved, "live_slots": live, "wasted_slots": reserved - live}
+
+
+def shared_prefix_groups(tables, lens, block_size: int, min_group_seqs: int = 2,
+                         min_shared_blocks: int = 1, max_groups: int = 64):
+    """Groups of consecutive sequences that share the leading blocks of their
+    tables, for the shared-prefix decode (sequences forked from one prompt
+    point their tables at the same blocks: "PagedAttention" ops page, At a
+    glance and How it works).  Returns (group_start, group_shared_blocks) with
+    len(group_start) == len(group_shared_blocks) + 1.
+
+    The rule, taken from the batch order: a group starts at sequence i and
+    takes i + 1, i + 2, ... as long as the leading table entries that all of
+    them have in common with row i, counting only blocks full in every one of
+    them, number at least ``min_shared_blocks``; it is kept when it has at
+    least ``min_group_seqs`` sequences, otherwise the walk moves on to i + 1.
+    Kept groups that are not back to back get a group sharing nothing between
+    them; groups past ``max_groups`` entries are dropped."""
+    n = len(lens)
+    width = len(tables[0]) if n else 0
+
+    def full(b):
+        return min(max(int(lens[b]), 0) // block_size, width)
+
+    kept = []
+    i = 0
+    while i < n and len(kept) < max_groups:
+        common = full(i)
+        j = i + 1
+        while j < n:
+            k = 0
+            limit = min(common, full(j))
+            while k < limit and tables[j][k] == tables[i][k]:
+                k += 1
+            if k < min_shared_blocks:
+                break
+            common = k
+            j += 1
+        if j - i >= min_group_seqs and common >= min_shared_blocks:
+            kept.append((i, j, common))
+            i = j
+        else:
+            i += 1
+    starts, shared, end = [], [], 0
+    for a, b, c in kept:
+        gap = bool(shared) and a != end
+        if len(shared) + (2 if gap else 1) > max_groups:
+            break
+        if gap:
+            starts.append(end)
+            shared.append(0)
+        starts.append(a)
+        shared.append(c)
+        end = b
+    starts.append(end)
+    return starts, shared

@@ -21,7 +21,9 @@ from ._lib import PkvError, PoolExhausted  # noqa: F401
 __all__ = [
     "paged_kv_append", "copy_blocks", "swap_blocks", "paged_attention_decode",
     "paged_attention_workspace_bytes",
-    "paged_attention_decode_static_scratch", "paged_attention_prefill", "Pool",
+    "paged_attention_decode_static_scratch", "paged_attention_prefill",
+    "paged_attention_decode_shared_prefix", "paged_attention_shared_prefix_workspace_bytes",
+    "shared_prefix_groups", "Pool",
     "PkvError", "PoolExhausted", "launch_count", "selftest_wait_timeout", "cache_desc",
 ]
 
@@ -173,6 +175,82 @@ def paged_attention_decode_static_scratch(out, q, k_cache, v_cache, block_tables
         ctypes.c_float(scale), int(partition_size), _dev(err_flag, "err_flag", torch.int32),
         _stream(stream)))
     return out
+
+
+def _group_arrays(group_start, group_shared_blocks):
+    gs = np.ascontiguousarray(group_start, dtype=np.int32)
+    gb = np.ascontiguousarray(group_shared_blocks, dtype=np.int32)
+    n = len(gb)
+    if gs.ndim != 1 or gb.ndim != 1 or len(gs) != n + 1:
+        raise PkvError(1, "group_start must have one entry more than group_shared_blocks")
+    return gs, gb, n
+
+
+def _ptr_np(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a.size else None
+
+
+def paged_attention_shared_prefix_workspace_bytes(k_cache, num_seqs: int, num_heads: int,
+                                                  max_blocks_per_seq: int, group_start,
+                                                  group_shared_blocks) -> int:
+    desc = cache_desc(k_cache)
+    gs, gb, n = _group_arrays(group_start, group_shared_blocks)
+    return int(_lib.load().paged_attention_shared_prefix_workspace_bytes(
+        ctypes.byref(desc), num_seqs, num_heads, max_blocks_per_seq, _ptr_np(gs), _ptr_np(gb), n))
+
+
+def paged_attention_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens,
+                                         scale, group_start, group_shared_blocks, workspace=None,
+                                         err_flag=None, stream=None):
+    """paged_attention_decode for a batch in which each group of consecutive
+    sequences group_start[i] .. group_start[i+1]-1 shares the first
+    group_shared_blocks[i] blocks of its tables (host int sequences; see
+    shared_prefix_groups).  The shared blocks are attended once per 128 query
+    rows on the tensor cores.  `workspace` (uint8 CUDA tensor, 256-byte
+    aligned) is allocated with torch when not given.  Returns `out`."""
+    torch = _torch()
+    desc = cache_desc(k_cache)
+    B, H, D = q.shape
+    if tuple(out.shape) != (B, H, D) or out.dtype != q.dtype or q.dtype != k_cache.dtype:
+        raise PkvError(1, "q and out must be [B, H, D] of the cache dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise PkvError(1, "block_tables must be [B, MB] and context_lens [B]")
+    MB = int(block_tables.shape[1])
+    gs, gb, n = _group_arrays(group_start, group_shared_blocks)
+    if workspace is None:
+        need = paged_attention_shared_prefix_workspace_bytes(k_cache, B, H, MB, gs, gb)
+        if need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _lib.check(_lib.load().paged_attention_decode_shared_prefix(
+        ctypes.byref(desc), _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"),
+        _dev(v_cache, "v_cache"), _dev(block_tables, "block_tables", torch.int32), MB,
+        _dev(context_lens, "context_lens", torch.int32), B, H, ctypes.c_float(scale), _ptr_np(gs),
+        _ptr_np(gb), n, _dev(workspace, "workspace"), ws_bytes,
+        _dev(err_flag, "err_flag", torch.int32), _stream(stream)))
+    return out
+
+
+def shared_prefix_groups(block_tables, context_lens, block_size: int, min_group_seqs: int = 2,
+                         min_shared_blocks: int = 1, max_groups: int = 64):
+    """(group_start, group_shared_blocks) for paged_attention_decode_shared_prefix
+    from host copies (numpy int32) of a batch's block tables [B, MB] and lengths
+    [B]: runs of consecutive sequences whose tables start with the same full
+    blocks (pkv_shared_prefix_groups)."""
+    tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    if tables.ndim != 2 or lens.shape != (tables.shape[0],):
+        raise PkvError(1, "block_tables must be [B, MB] and context_lens [B]")
+    B, MB = tables.shape
+    starts = np.zeros(max_groups + 1, dtype=np.int32)
+    shared = np.zeros(max(1, max_groups), dtype=np.int32)
+    n = ctypes.c_int32()
+    _lib.check(_lib.load().pkv_shared_prefix_groups(
+        _ptr_np(tables), B, max(1, MB), _ptr_np(lens), block_size, min_group_seqs,
+        min_shared_blocks, max_groups, starts.ctypes.data_as(ctypes.c_void_p),
+        shared.ctypes.data_as(ctypes.c_void_p), ctypes.byref(n)))
+    k = n.value
+    return starts[:k + 1], shared[:k]
 
 
 def paged_attention_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start,

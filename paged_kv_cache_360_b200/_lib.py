@@ -26,10 +26,11 @@ STATIC_SCRATCH_BYTES = 16 << 20
 EXPORTS = (
     "paged_kv_append", "copy_blocks", "swap_blocks", "paged_attention_workspace_bytes", "paged_attention_decode",
     "paged_attention_decode_static_scratch", "paged_attention_prefill",
+    "paged_attention_decode_shared_prefix", "paged_attention_shared_prefix_workspace_bytes",
     "pkv_pool_create", "pkv_pool_destroy", "pkv_seq_new", "pkv_seq_fork", "pkv_seq_reserve",
     "pkv_seq_reserve_tokens", "pkv_seq_new_cached", "pkv_pool_reserve_batch",
     "pkv_seq_cow", "pkv_seq_free", "pkv_seq_swap_out", "pkv_seq_swap_in", "pkv_seq_len", "pkv_seq_block_table", "pkv_pool_block_tables",
-    "pkv_pool_refcount", "pkv_pool_free_list", "pkv_pool_stats",
+    "pkv_pool_refcount", "pkv_pool_free_list", "pkv_pool_stats", "pkv_shared_prefix_groups",
     "pkv_launch_count", "pkv_last_error", "pkv_status_string", "pkv_selftest_wait_timeout",
 )
 
@@ -85,6 +86,11 @@ def load():
                                                                i32, i32, ctypes.c_float, i32, p, p]),
                 "paged_attention_prefill": (st, [P(CacheDesc), p, p, p, p, p, i32, p, p, i32, i32,
                                                  i32, ctypes.c_float, p, p]),
+                "paged_attention_decode_shared_prefix": (st, [P(CacheDesc), p, p, p, p, p, i32, p, i32,
+                                                              i32, ctypes.c_float, p, p, i32, p, sz,
+                                                              p, p]),
+                "paged_attention_shared_prefix_workspace_bytes": (sz, [P(CacheDesc), i32, i32, i32, p,
+                                                                       p, i32]),
                 "pkv_pool_create": (st, [i32, i32, p, P(p)]),
                 "pkv_pool_destroy": (None, [p]),
                 "pkv_seq_new": (st, [p, P(i32)]),
@@ -103,6 +109,7 @@ def load():
                 "pkv_pool_refcount": (st, [p, i32, P(i32)]),
                 "pkv_pool_free_list": (st, [p, p, i32, P(i32)]),
                 "pkv_pool_stats": (st, [p, P(Stats)]),
+                "pkv_shared_prefix_groups": (st, [p, i32, i32, p, i32, i32, i32, i32, p, p, P(i32)]),
                 "pkv_launch_count": (ctypes.c_uint64, []),
                 "pkv_last_error": (ctypes.c_char_p, []),
                 "pkv_status_string": (ctypes.c_char_p, [st]),

@@ -1,0 +1,83 @@
+// pkv_cascade.cuh -- the table of shared-prefix groups that the shared-prefix
+// decode hands to its kernels as a kernel parameter.
+//
+// "PagedAttention" ops page, At a glance and How it works: sequences that share
+// a prompt point their block tables at the same physical blocks.  A group is a
+// run of consecutive sequences of the batch whose first `shared_tokens /
+// block_size` table entries are the same blocks; the decode attends every
+// query of the group to those blocks in one tensor-core pass (prefix_kernel)
+// and each sequence's own tokens with the balanced decode, and folds the two
+// into one softmax by log-sum-exp.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pkv.h"
+
+namespace pkv {
+
+constexpr int kMaxGroups = 64;  // groups per call (the table is a kernel parameter)
+constexpr int kPrefixRows = 128;  // query rows of one prefix tile: 128 / g sequences x g heads
+constexpr int kPrefixKv = 128;    // kv tokens of one prefix kv tile
+
+struct CascadeGroups {
+    int32_t num_groups;
+    int32_t tiles_per_item;                 // kv tiles of one prefix work item (1 or 2)
+    int32_t start[kMaxGroups + 1];          // group i = sequences start[i] .. start[i+1]-1
+    int32_t shared_tokens[kMaxGroups];      // tokens of the shared blocks (a multiple of bs)
+    int32_t chunks[kMaxGroups];             // prefix partials per (sequence, head)
+    int32_t pre_base[kMaxGroups];           // first partial slot of the group
+    int32_t item_base[kMaxGroups + 1];      // prefix work items before group i
+    float* pre_o;                           // [slot][D]   un-normalised partial O
+    float* pre_ml;                          // [slot][2]   partial (m, l), m in base-2 units
+};
+
+// Partial slot of (sequence b of group i, query head h, chunk c).
+__host__ __device__ __forceinline__ int64_t prefix_slot(const CascadeGroups& cg, int i, int b,
+                                                         int num_heads, int h, int c) {
+    return static_cast<int64_t>(cg.pre_base[i]) +
+           (static_cast<int64_t>(b - cg.start[i]) * num_heads + h) * cg.chunks[i] + c;
+}
+
+// Index of the group holding sequence b, or -1.
+__device__ __forceinline__ int group_of(const CascadeGroups& cg, int b) {
+    int lo = 0, hi = cg.num_groups;  // first group whose end is past b
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (cg.start[mid + 1] <= b) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo < cg.num_groups && cg.start[lo] <= b ? lo : -1;
+}
+
+// Tokens at the start of sequence b that the prefix kernel attends (0 outside
+// a group).
+__device__ __forceinline__ int shared_begin(const CascadeGroups& cg, int b) {
+    const int i = group_of(cg, b);
+    return i < 0 ? 0 : cg.shared_tokens[i];
+}
+
+// Stand-in for the group table in the plain decode's kernels.
+struct NoGroups {
+    int32_t unused;
+};
+
+// Prefix work items (1 kv tile each) from which an item takes 2 kv tiles.
+constexpr int kPrefixTwoTilesFrom = 296;
+
+// Lay out the group table for these shapes from the caller's host arrays
+// (group_start [num_groups + 1], group_shared_blocks [num_groups]); *slots =
+// prefix partial slots.  Errors are recorded for pkv_last_error().
+pkv_status plan_groups(const pkv_cache_desc* desc, int32_t num_seqs, int32_t num_heads,
+                       int32_t max_blocks_per_seq, const int32_t* group_start,
+                       const int32_t* group_shared_blocks, int32_t num_groups, CascadeGroups* cg,
+                       int64_t* slots);
+
+// The prefix kernel over every work item of `cg` (pkv_cascade.cu).
+pkv_status launch_prefix(const pkv_cache_desc* desc, const void* q, const void* k_cache,
+                         const void* v_cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                         int32_t num_seqs, int32_t num_heads, float scale, const CascadeGroups& cg,
+                         int32_t* err_flag, cudaStream_t stream);
+
+}  // namespace pkv

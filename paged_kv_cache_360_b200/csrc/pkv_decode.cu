@@ -43,10 +43,12 @@
 
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 
 #include "pkv.h"
 #include "pkv_attend.cuh"
+#include "pkv_cascade.cuh"
 #include "pkv_host.cuh"
 #include "pkv_internal.h"
 #include "pkv_ptx.cuh"
@@ -373,12 +375,13 @@ struct BalancedArgs {
     int32_t group;
     int32_t max_blocks_per_seq;
     int32_t num_blocks;
+    int32_t max_len;  // max_blocks_per_seq * block_size
     float scale_log2;
 };
 
 struct SegDesc {
     int32_t b, hk, first, n;  // CTA-local index of the first unit, unit count
-    int32_t blk0, len, flags, pad;
+    int32_t blk0, len, flags, beg;  // beg: first token the segment's units count from
 };
 
 // The balanced kernel streams 16-token units: a block of 32 tokens is two units
@@ -461,15 +464,29 @@ __device__ __forceinline__ void load_unit(const CUtensorMap* tm_k, const CUtenso
 struct Chunk {
     int b, hk, u0, cnt;   // sequence, kv head, first unit within (b, hk), units
     int len, nu;          // the sequence's length and its units per kv head
+    int beg;              // first token of unit 0 (after the shared prefix, if any)
     int seg_start;        // the chunk opens a segment of seg_len units
     int seg_len;
     int phys;             // this lane's physical block
 };
 
-template <typename T, int D, int BS>
+// With CASCADE, sequences of a shared-prefix group attend here only to their
+// own tokens (from the group's shared_tokens on; units count from there), and
+// the segment that starts a (b, hk) folds in the prefix kernel's partials of
+// those rows (CascadeGroups: written before this kernel starts).
+template <bool CASCADE>
+using GroupsOf = typename std::conditional<CASCADE, CascadeGroups, NoGroups>::type;
+
+template <bool CASCADE>
+__device__ __forceinline__ int first_token(const GroupsOf<CASCADE>& cg, int b) {
+    if constexpr (CASCADE) return shared_begin(cg, b);
+    else return 0;
+}
+
+template <typename T, int D, int BS, bool CASCADE>
 __global__ void __launch_bounds__(kBalancedThreads, 2)
 balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                const BalancedArgs a) {
+                const BalancedArgs a, const __grid_constant__ GroupsOf<CASCADE> cg) {
     using G = UnitGeom<D>;
     constexpr int R = BS / 16;  // units per block
     extern __shared__ uint8_t smem_raw[];
@@ -512,8 +529,9 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     for (int b = b_lo; b < b_hi; ++b) {
         const int raw = __ldg(a.context_lens + b);
         const int L = clamp_len(raw, max_len);
-        if (raw != L && c == 0) flag(a.err_flag, PKV_DEVERR_BAD_CONTEXT_LEN);
-        mine += (L + 15) / 16;
+        const int beg = first_token<CASCADE>(cg, b);
+        if ((raw != L || L < beg) && c == 0) flag(a.err_flag, PKV_DEVERR_BAD_CONTEXT_LEN);
+        mine += (max(L - beg, 0) + 15) / 16;
     }
     long long incl = mine;
 #pragma unroll
@@ -542,7 +560,8 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     if (u0 < u1 && mine > 0 && excl * Hkv <= u0 && u0 < (excl + mine) * Hkv) {
         long long p = excl;
         for (int b = b_lo; b < b_hi; ++b) {
-            const int nu = (clamp_len(__ldg(a.context_lens + b), max_len) + 15) / 16;
+            const int nu =
+                (max(clamp_len(__ldg(a.context_lens + b), max_len) - first_token<CASCADE>(cg, b), 0) + 15) / 16;
             if (u0 < (p + nu) * Hkv) {
                 const long long r = u0 - p * Hkv;
                 s_start[0] = b;
@@ -585,7 +604,8 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const uint64_t policy = l2_evict_first_policy();
         int b = s_start[0], hk = s_start[1], ub = s_start[2];  // walk cursor
         int len = clamp_len(__ldg(a.context_lens + b), max_len);
-        int nu = (len + 15) / 16;
+        int beg = first_token<CASCADE>(cg, b);
+        int nu = (max(len - beg, 0) + 15) / 16;
         // raw, clamped only when used, so the load does not stall the warp here
         int len_next_raw = b + 1 < B ? __ldg(a.context_lens + b + 1) : 0;
         int walked = 0;  // units already assigned to chunks
@@ -598,11 +618,13 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     hk = 0;
                     ++b;
                     len = clamp_len(len_next_raw, max_len);
-                    while (len == 0 && b + 1 < B) {
+                    beg = first_token<CASCADE>(cg, b);
+                    while (len <= beg && b + 1 < B) {
                         ++b;
                         len = clamp_len(__ldg(a.context_lens + b), max_len);
+                        beg = first_token<CASCADE>(cg, b);
                     }
-                    nu = (len + 15) / 16;
+                    nu = (max(len - beg, 0) + 15) / 16;
                     len_next_raw = b + 1 < B ? __ldg(a.context_lens + b + 1) : 0;
                 }
             }
@@ -611,6 +633,7 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             ch.u0 = ub;
             ch.len = len;
             ch.nu = nu;
+            ch.beg = beg;
             ch.cnt = min(32, min(nu - ub, n_units - walked));
             if (ch.cnt <= 0) return false;  // lengths changed under the kernel
             ch.seg_start = ub == 0 || walked == 0;
@@ -618,7 +641,7 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             // the entries are checked when they are used, so the loads stay in flight
             ch.phys = lane < ch.cnt
                           ? __ldg(a.block_tables + static_cast<int64_t>(b) * a.max_blocks_per_seq +
-                                  (ub + lane) / R)
+                                  beg / BS + (ub + lane) / R)
                           : 0;
             ub += ch.cnt;
             walked += ch.cnt;
@@ -647,6 +670,7 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         d.n = cur.seg_len;
                         d.blk0 = cur.u0;
                         d.len = cur.len;
+                        d.beg = cur.beg;
                         d.flags = (cur.u0 == 0 ? kMetaBegins : 0) |
                                   (cur.u0 + cur.seg_len == cur.nu ? kMetaEnds : 0) |
                                   (i == 0 ? kSegFirstInCta : 0);
@@ -734,6 +758,15 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const int sb = smeta[0], shk = smeta[1];
             const bool complete = (flags & (kMetaBegins | kMetaEnds)) == (kMetaBegins | kMetaEnds);
             const int64_t pslot = static_cast<int64_t>(c) * 2 + ((flags & kSegFirstInCta) ? 0 : 1);
+            // The segment that starts a grouped sequence's own tokens also
+            // takes the prefix kernel's partials of its rows, after the warps'.
+            int pgrp = -1;
+            if constexpr (CASCADE) {
+                if (flags & kMetaBegins) {
+                    pgrp = group_of(cg, sb);
+                    if (pgrp >= 0 && cg.shared_tokens[pgrp] == 0) pgrp = -1;
+                }
+            }
             // Row by row: the weights 2^(m_w - M) once per row, then four columns
             // per lane (M = max_w m_w; acc = sum_w 2^(m_w - M) o_w; den likewise).
             for (int r = 0; r < group; ++r) {
@@ -742,6 +775,15 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 for (int w = 0; w < kConsumerWarps; ++w) {
                     mw[w] = mm[w * group + r];
                     M = fmaxf(M, mw[w]);
+                }
+                int64_t pre0 = 0;
+                int nchunk = 0;
+                if constexpr (CASCADE) {
+                    if (pgrp >= 0) {
+                        nchunk = cg.chunks[pgrp];
+                        pre0 = prefix_slot(cg, pgrp, sb, a.num_heads, shk * group + r, 0);
+                        for (int k = 0; k < nchunk; ++k) M = fmaxf(M, cg.pre_ml[(pre0 + k) * 2]);
+                    }
                 }
                 float f[kConsumerWarps], den = 0.f;
 #pragma unroll
@@ -759,6 +801,18 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         acc.y += f[w] * o.y;
                         acc.z += f[w] * o.z;
                         acc.w += f[w] * o.w;
+                    }
+                    if constexpr (CASCADE) {
+                        for (int k = 0; k < nchunk; ++k) {
+                            const float2 ml_k = *reinterpret_cast<const float2*>(cg.pre_ml + (pre0 + k) * 2);
+                            const float fk = ml_k.x == -INFINITY ? 0.f : exp2_approx(ml_k.x - M);
+                            const float4 o = *reinterpret_cast<const float4*>(cg.pre_o + (pre0 + k) * D + d0);
+                            acc.x += fk * o.x;
+                            acc.y += fk * o.y;
+                            acc.z += fk * o.z;
+                            acc.w += fk * o.w;
+                            den += fk * ml_k.y;
+                        }
                     }
                     if (complete) {
                         const float inv = den > 0.f ? 1.f / den : 0.f;
@@ -841,7 +895,7 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
             const uint32_t kst = base + s * G::kStageBytes;
             attend_16<T, D>(st, qa, kst, kst + G::kTileBytes, G::kHalfBytes, 0,
-                            (d.blk0 + (u - d.first)) * 16, d.len, a.scale_log2, lane);
+                            d.beg + (d.blk0 + (u - d.first)) * 16, d.len, a.scale_log2, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_empty + 8 * s);
         }
@@ -868,8 +922,11 @@ constexpr int kReduceThreads = 128;
 constexpr int kChainWindow = 32;  // chains up to this many CTAs long are found in one round
 constexpr int kShortChain = 4;    // chains up to this long are merged from registers
 
-template <typename T, int D>
-__global__ void __launch_bounds__(kReduceThreads) balanced_reduce_kernel(const BalancedArgs a) {
+// With CASCADE, a grouped sequence with no tokens of its own (all of its
+// context is the shared prefix) gets the prefix kernel's partials merged here.
+template <typename T, int D, bool CASCADE>
+__global__ void __launch_bounds__(kReduceThreads)
+    balanced_reduce_kernel(const BalancedArgs a, const __grid_constant__ GroupsOf<CASCADE> cg) {
     __shared__ int s_meta[2 + kChainWindow][3];  // own slots 0 and 1, then slot 0 of c+1 ..
     __shared__ int s_len[2];
     const int c = blockIdx.x;
@@ -882,10 +939,15 @@ __global__ void __launch_bounds__(kReduceThreads) balanced_reduce_kernel(const B
 
     // The lengths are an input of the whole step (ready before the decode
     // started), so they are read before waiting for the decode's results.
+    // tokens the balanced kernel attends for sequence b (lengths clamped as there)
+    auto own_tokens = [&](int b) {
+        const int L = clamp_len(__ldg(a.context_lens + b), a.max_len);
+        return L - first_token<CASCADE>(cg, b);
+    };
     bool empty_seq[4] = {false, false, false, false};
     {
         int k = 0;
-        for (int b = c; b < a.num_seqs && k < 4; b += grid, ++k) empty_seq[k] = __ldg(a.context_lens + b) <= 0;
+        for (int b = c; b < a.num_seqs && k < 4; b += grid, ++k) empty_seq[k] = own_tokens(b) <= 0;
     }
 
     pdl_wait_primary();  // the decode's partials and descriptors are visible after this
@@ -1008,13 +1070,40 @@ __global__ void __launch_bounds__(kReduceThreads) balanced_reduce_kernel(const B
         }
     }
 
-    // sequences with no tokens: zeros (context lengths <= 0 count as empty)
+    // sequences with no tokens: zeros (context lengths <= 0 count as empty);
+    // with CASCADE, a grouped sequence whose tokens are all shared: its prefix
+    // partials, merged in chunk order
     int k = 0;
     for (int b = c; b < a.num_seqs; b += grid, ++k) {
-        const bool empty = k < 4 ? empty_seq[k] : __ldg(a.context_lens + b) <= 0;
+        const bool empty = k < 4 ? empty_seq[k] : own_tokens(b) <= 0;
         if (!empty) continue;
         T* o = static_cast<T*>(a.out) + static_cast<int64_t>(b) * a.num_heads * D;
-        for (int idx = tid; idx < a.num_heads * D; idx += kReduceThreads) o[idx] = Pack<T>::one(0.f);
+        int pgrp = -1;
+        if constexpr (CASCADE) {
+            pgrp = group_of(cg, b);
+            if (pgrp >= 0 && (cg.shared_tokens[pgrp] == 0 || __ldg(a.context_lens + b) <= 0)) pgrp = -1;
+        }
+        if (pgrp < 0) {
+            for (int idx = tid; idx < a.num_heads * D; idx += kReduceThreads) o[idx] = Pack<T>::one(0.f);
+            continue;
+        }
+        if constexpr (CASCADE) {
+            const int nchunk = cg.chunks[pgrp];
+            for (int idx = tid; idx < a.num_heads * D; idx += kReduceThreads) {
+                const int h = idx / D, d = idx - h * D;
+                const int64_t p0 = prefix_slot(cg, pgrp, b, a.num_heads, h, 0);
+                float M = -INFINITY;
+                for (int q = 0; q < nchunk; ++q) M = fmaxf(M, cg.pre_ml[(p0 + q) * 2]);
+                float acc = 0.f, den = 0.f;
+                for (int q = 0; q < nchunk; ++q) {
+                    const float mq = cg.pre_ml[(p0 + q) * 2];
+                    const float f = mq == -INFINITY ? 0.f : exp2_approx(mq - M);
+                    acc += f * cg.pre_o[(p0 + q) * D + d];
+                    den += f * cg.pre_ml[(p0 + q) * 2 + 1];
+                }
+                o[idx] = Pack<T>::one(den > 0.f ? acc / den : 0.f);
+            }
+        }
     }
 }
 
@@ -1046,7 +1135,7 @@ pkv_status encode_pool_map(CUtensorMap* tm, const void* pool, const pkv_cache_de
 
 template <typename T, int D, int BS, bool SPLIT>
 struct FixedTag {};
-template <typename T, int D, int BS>
+template <typename T, int D, int BS, bool CASCADE>
 struct BalancedTag {};
 
 template <typename T, int D, int BS>
@@ -1107,8 +1196,8 @@ pkv_status balanced_grid(int group, int* grid_out, int* smem_out) {
             return PKV_OK;
         }
     }
-    auto k = balanced_kernel<T, D, BS>;
-    cudaError_t e = opt_in_smem<BalancedTag<T, D, BS>>(reinterpret_cast<const void*>(k));
+    auto k = balanced_kernel<T, D, BS, false>;
+    cudaError_t e = opt_in_smem<BalancedTag<T, D, BS, false>>(reinterpret_cast<const void*>(k));
     if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
     int dev = 0, sms = 0, per_sm = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
@@ -1123,11 +1212,20 @@ pkv_status balanced_grid(int group, int* grid_out, int* smem_out) {
     return PKV_OK;
 }
 
-template <typename T, int D, int BS>
+// The cascade kernel has the same threads, shared memory and register cap
+// (__launch_bounds__(.., 2)) as the plain one, so the same grid (and workspace
+// layout) serves both.
+template <typename T, int D, int BS, bool CASCADE>
 pkv_status launch_balanced(const CUtensorMap& tk, const CUtensorMap& tv, const BalancedArgs& a,
-                           int grid, int smem, cudaStream_t stream) {
-    cudaError_t e = launch_dependent(balanced_kernel<T, D, BS>, dim3(grid), dim3(kBalancedThreads), smem,
-                                     stream, tk, tv, a);
+                           const GroupsOf<CASCADE>& cg, int grid, int smem, cudaStream_t stream) {
+    cudaError_t e;
+    if constexpr (CASCADE) {
+        e = opt_in_smem<BalancedTag<T, D, BS, true>>(
+            reinterpret_cast<const void*>(balanced_kernel<T, D, BS, true>));
+        if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+    }
+    e = launch_dependent(balanced_kernel<T, D, BS, CASCADE>, dim3(grid), dim3(kBalancedThreads), smem,
+                         stream, tk, tv, a, cg);
     note_launches(1);
     if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
     cudaLaunchConfig_t cfg = {};
@@ -1139,7 +1237,7 @@ pkv_status launch_balanced(const CUtensorMap& tk, const CUtensorMap& tv, const B
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, balanced_reduce_kernel<T, D>, a);
+    e = cudaLaunchKernelEx(&cfg, balanced_reduce_kernel<T, D, CASCADE>, a, cg);
     note_launches(1);
     if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
     return PKV_OK;
@@ -1175,7 +1273,14 @@ template <typename T, int D, int BS>
 struct RunBalanced {
     static pkv_status run(const CUtensorMap& tk, const CUtensorMap& tv, const BalancedArgs& a,
                           int grid, int smem, cudaStream_t st) {
-        return launch_balanced<T, D, BS>(tk, tv, a, grid, smem, st);
+        return launch_balanced<T, D, BS, false>(tk, tv, a, NoGroups{0}, grid, smem, st);
+    }
+};
+template <typename T, int D, int BS>
+struct RunCascade {
+    static pkv_status run(const CUtensorMap& tk, const CUtensorMap& tv, const BalancedArgs& a,
+                          const CascadeGroups& cg, int grid, int smem, cudaStream_t st) {
+        return launch_balanced<T, D, BS, true>(tk, tv, a, cg, grid, smem, st);
     }
 };
 
@@ -1229,15 +1334,15 @@ extern "C" size_t paged_attention_workspace_bytes(const pkv_cache_desc* desc, in
     return balanced_workspace(grid, group, desc->head_dim);
 }
 
-extern "C" pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* out, const void* q,
-                                             const void* k_cache, const void* v_cache,
-                                             const int32_t* block_tables,
-                                             int32_t max_blocks_per_seq,
-                                             const int32_t* context_lens, int32_t num_seqs,
-                                             int32_t num_heads, float scale,
-                                             int32_t partition_size, void* workspace,
-                                             size_t workspace_bytes, int32_t* err_flag,
-                                             void* stream) {
+namespace pkv {
+namespace {
+
+// Host checks shared by the decode entry points (nothing is enqueued when they
+// fail); num_seqs == 0 passes and means nothing to do.
+pkv_status check_decode_args(const pkv_cache_desc* desc, const void* out, const void* q,
+                             const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                             int32_t max_blocks_per_seq, const int32_t* context_lens,
+                             int32_t num_seqs, int32_t num_heads, float scale) {
     pkv_status st = check_desc(desc);
     if (st != PKV_OK) return st;
     if (num_seqs < 0 || num_heads <= 0 || max_blocks_per_seq <= 0)
@@ -1251,8 +1356,8 @@ extern "C" pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* o
                     "paged_attention_decode: q, out and pools must be 16-byte aligned");
     if (num_heads % desc->num_kv_heads != 0)
         return fail(PKV_ERR_INVALID_ARG, "num_heads must be a multiple of num_kv_heads");
-    const int32_t group = num_heads / desc->num_kv_heads;
-    if (group > 16) return fail(PKV_ERR_UNSUPPORTED, "num_heads / num_kv_heads must be <= 16");
+    if (num_heads / desc->num_kv_heads > 16)
+        return fail(PKV_ERR_UNSUPPORTED, "num_heads / num_kv_heads must be <= 16");
     if (!(scale == scale) || scale == INFINITY || scale == -INFINITY)
         return fail(PKV_ERR_INVALID_ARG, "scale must be finite");
     if (static_cast<int64_t>(max_blocks_per_seq) * desc->block_size > INT32_MAX / 2)
@@ -1260,6 +1365,25 @@ extern "C" pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* o
     if (static_cast<int64_t>(num_seqs) * max_blocks_per_seq * desc->num_kv_heads > INT32_MAX)
         return fail(PKV_ERR_UNSUPPORTED,
                     "num_seqs * max_blocks_per_seq * num_kv_heads must be < 2^31");
+    return PKV_OK;
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* out, const void* q,
+                                             const void* k_cache, const void* v_cache,
+                                             const int32_t* block_tables,
+                                             int32_t max_blocks_per_seq,
+                                             const int32_t* context_lens, int32_t num_seqs,
+                                             int32_t num_heads, float scale,
+                                             int32_t partition_size, void* workspace,
+                                             size_t workspace_bytes, int32_t* err_flag,
+                                             void* stream) {
+    pkv_status st = check_decode_args(desc, out, q, k_cache, v_cache, block_tables,
+                                      max_blocks_per_seq, context_lens, num_seqs, num_heads, scale);
+    if (st != PKV_OK || num_seqs == 0) return st;
+    const int32_t group = num_heads / desc->num_kv_heads;
     if (partition_size < 0 || (partition_size > 0 && partition_size % desc->block_size != 0))
         return fail(PKV_ERR_INVALID_ARG,
                     "partition_size must be 0 or a positive multiple of block_size");
@@ -1292,6 +1416,7 @@ extern "C" pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* o
         a.group = group;
         a.max_blocks_per_seq = max_blocks_per_seq;
         a.num_blocks = desc->num_blocks;
+        a.max_len = max_blocks_per_seq * desc->block_size;
         a.scale_log2 = scale * kLog2e;
         return dispatch<RunBalanced>(desc, tk, tv, a, grid, smem, s);
     }
@@ -1331,6 +1456,87 @@ extern "C" pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* o
     if ((st = encode_pool_map(&tk, k_cache, desc, desc->block_size)) != PKV_OK) return st;
     if ((st = encode_pool_map(&tv, v_cache, desc, desc->block_size)) != PKV_OK) return st;
     return dispatch<RunFixed>(desc, tk, tv, a, num_seqs, split, s);
+}
+
+// ------------------------------------------------------ shared-prefix decode
+
+namespace pkv {
+namespace {
+
+size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" size_t paged_attention_shared_prefix_workspace_bytes(
+    const pkv_cache_desc* desc, int32_t num_seqs, int32_t num_heads, int32_t max_blocks_per_seq,
+    const int32_t* group_start, const int32_t* group_shared_blocks, int32_t num_groups) {
+    const size_t plain = paged_attention_workspace_bytes(desc, num_seqs, num_heads, max_blocks_per_seq, 0);
+    if (plain == 0) return 0;
+    CascadeGroups cg;
+    int64_t slots = 0;
+    if (plan_groups(desc, num_seqs, num_heads, max_blocks_per_seq, group_start, group_shared_blocks,
+                    num_groups, &cg, &slots) != PKV_OK)
+        return 0;
+    return align256(plain) + static_cast<size_t>(slots) * (desc->head_dim + 2) * sizeof(float);
+}
+
+extern "C" pkv_status paged_attention_decode_shared_prefix(
+    const pkv_cache_desc* desc, void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+    int32_t num_seqs, int32_t num_heads, float scale, const int32_t* group_start,
+    const int32_t* group_shared_blocks, int32_t num_groups, void* workspace, size_t workspace_bytes,
+    int32_t* err_flag, void* stream) {
+    pkv_status st = check_decode_args(desc, out, q, k_cache, v_cache, block_tables,
+                                      max_blocks_per_seq, context_lens, num_seqs, num_heads, scale);
+    if (st != PKV_OK || num_seqs == 0) return st;
+    CascadeGroups cg;
+    int64_t slots = 0;
+    if ((st = plan_groups(desc, num_seqs, num_heads, max_blocks_per_seq, group_start,
+                          group_shared_blocks, num_groups, &cg, &slots)) != PKV_OK)
+        return st;
+    const int32_t group = num_heads / desc->num_kv_heads;
+    int grid = 0, smem = 0;
+    if ((st = dispatch<GridOf>(desc, static_cast<int>(group), &grid, &smem)) != PKV_OK) return st;
+    const size_t plain = balanced_workspace(grid, group, desc->head_dim);
+    const size_t need = align256(plain) + static_cast<size_t>(slots) * (desc->head_dim + 2) * sizeof(float);
+    if (!workspace || workspace_bytes < need)
+        return fail(PKV_ERR_WORKSPACE_TOO_SMALL, "paged_attention_decode_shared_prefix: workspace too small");
+    if (!aligned(workspace, 256))
+        return fail(PKV_ERR_INVALID_ARG,
+                    "paged_attention_decode_shared_prefix: workspace must be 256-byte aligned");
+    if (cg.item_base[cg.num_groups] == 0)  // no group shares a block: the plain decode
+        return paged_attention_decode(desc, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                      context_lens, num_seqs, num_heads, scale, 0, workspace,
+                                      workspace_bytes, err_flag, stream);
+    cg.pre_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256(plain));
+    cg.pre_ml = cg.pre_o + slots * desc->head_dim;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = launch_prefix(desc, q, k_cache, v_cache, block_tables, max_blocks_per_seq, num_seqs,
+                            num_heads, scale, cg, err_flag, s)) != PKV_OK)
+        return st;
+    CUtensorMap tk, tv;
+    if ((st = encode_pool_map(&tk, k_cache, desc, 16)) != PKV_OK) return st;
+    if ((st = encode_pool_map(&tv, v_cache, desc, 16)) != PKV_OK) return st;
+    BalancedArgs a = {};
+    a.out = out;
+    a.q = q;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.ws_o = static_cast<float*>(workspace);
+    a.ws_ml = a.ws_o + static_cast<int64_t>(grid) * 2 * group * desc->head_dim;
+    a.ws_meta = reinterpret_cast<int32_t*>(a.ws_ml + static_cast<int64_t>(grid) * 2 * group * 2);
+    a.err_flag = err_flag;
+    a.num_seqs = num_seqs;
+    a.num_heads = num_heads;
+    a.num_kv_heads = desc->num_kv_heads;
+    a.group = group;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.num_blocks = desc->num_blocks;
+    a.max_len = max_blocks_per_seq * desc->block_size;
+    a.scale_log2 = scale * kLog2e;
+    return dispatch<RunCascade>(desc, tk, tv, a, cg, grid, smem, s);
 }
 
 // ------------------------------------------------ decode without allocation

@@ -476,3 +476,73 @@ extern "C" pkv_status pkv_pool_stats(const pkv_pool* pool, pkv_stats* st) {
     st->cached_blocks = static_cast<int64_t>(pool->cache.size());
     return PKV_OK;
 }
+
+// Groups for paged_attention_decode_shared_prefix from host copies of a
+// batch's block tables and lengths.  Walking the batch in order, a group
+// starts at sequence i and takes i + 1, i + 2, ... while the first entries
+// they have in common with row i (counting only blocks that are full in every
+// sequence taken so far) stay at least min_shared_blocks; it is kept when it
+// holds at least min_group_seqs sequences (else the walk moves on to i + 1).
+// Sequences outside every group are left out of group_start: they are decoded
+// as usual.  At most max_groups groups.
+extern "C" pkv_status pkv_shared_prefix_groups(const int32_t* block_tables, int32_t num_seqs,
+                                               int32_t max_blocks_per_seq,
+                                               const int32_t* context_lens, int32_t block_size,
+                                               int32_t min_group_seqs, int32_t min_shared_blocks,
+                                               int32_t max_groups, int32_t* group_start,
+                                               int32_t* group_shared_blocks, int32_t* num_groups) {
+    if (!num_groups || num_seqs < 0 || max_blocks_per_seq <= 0 || block_size <= 0 ||
+        min_group_seqs < 1 || min_shared_blocks < 1 || max_groups < 0)
+        return pkv::fail(PKV_ERR_INVALID_ARG, "pkv_shared_prefix_groups: bad sizes");
+    if (num_seqs > 0 && (!block_tables || !context_lens))
+        return pkv::fail(PKV_ERR_INVALID_ARG, "pkv_shared_prefix_groups: NULL tables or lengths");
+    if (max_groups > 0 && (!group_start || !group_shared_blocks))
+        return pkv::fail(PKV_ERR_INVALID_ARG, "pkv_shared_prefix_groups: NULL outputs");
+    auto full_blocks = [&](int32_t b) {
+        const int64_t f = context_lens[b] > 0 ? context_lens[b] / block_size : 0;
+        return static_cast<int32_t>(f < max_blocks_per_seq ? f : max_blocks_per_seq);
+    };
+    int32_t n = 0;
+    std::vector<int32_t> starts, ends, shared;
+    int32_t i = 0;
+    while (i < num_seqs && n < max_groups) {
+        const int32_t* row_i = block_tables + static_cast<int64_t>(i) * max_blocks_per_seq;
+        int32_t common = full_blocks(i);
+        int32_t j = i + 1;
+        for (; j < num_seqs; ++j) {
+            const int32_t* row_j = block_tables + static_cast<int64_t>(j) * max_blocks_per_seq;
+            int32_t lim = common < full_blocks(j) ? common : full_blocks(j);
+            int32_t k = 0;
+            while (k < lim && row_j[k] == row_i[k]) ++k;
+            if (k < min_shared_blocks) break;
+            common = k;
+        }
+        if (j - i >= min_group_seqs && common >= min_shared_blocks) {
+            starts.push_back(i);
+            ends.push_back(j);
+            shared.push_back(common);
+            ++n;
+            i = j;
+        } else {
+            ++i;
+        }
+    }
+    // Groups must be back to back in group_start; a gap between two groups
+    // becomes a group of its own that shares nothing.
+    int32_t out = 0;
+    for (int32_t g = 0; g < n; ++g) {
+        const bool gap = g > 0 && starts[g] != ends[g - 1];
+        if (out + (gap ? 2 : 1) > max_groups) break;
+        if (gap) {
+            group_start[out] = ends[g - 1];
+            group_shared_blocks[out] = 0;
+            ++out;
+        }
+        group_start[out] = starts[g];
+        group_shared_blocks[out] = shared[g];
+        ++out;
+        group_start[out] = ends[g];
+    }
+    *num_groups = out;
+    return PKV_OK;
+}

@@ -47,6 +47,7 @@
 #include "pkv_internal.h"
 #include "pkv_ptx.cuh"
 #include "pkv_tc.cuh"
+#include "pkv_wait.cuh"
 
 namespace pkv {
 namespace {
@@ -153,52 +154,6 @@ __device__ __forceinline__ uint32_t pack_pair(float lo, float hi) {
 
 __device__ __forceinline__ void flag(int32_t* err, int bit) {
     if (err) atomicOr(err, bit);
-}
-
-// Every wait below gives up after kWaitCycles SM cycles (about half a second,
-// defined with the other PTX wrappers): a protocol fault then costs each CTA a
-// bounded delay, never a hang.
-
-// Wait that also gives up when another role raised the abort word.
-// Warp-uniform: every lane of the calling warp must call it.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
-                                          volatile uint32_t* abort_word, int32_t* err) {
-    bool ok = false;
-    const long long t0 = clock64();
-    for (;;) {
-        if (mbar_test(bar, parity)) {
-            ok = true;
-            break;
-        }
-        if (*abort_word || clock64() - t0 > kWaitCycles) break;
-    }
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok && *abort_word == 0u) {
-        *abort_word = 1u;
-        if ((threadIdx.x & 31) == 0) flag(err, PKV_DEVERR_WAIT_TIMEOUT);
-    }
-    return ok;
-}
-
-// Single-thread variant (MMA issuer).
-__device__ __forceinline__ bool one_wait(uint32_t bar, uint32_t parity,
-                                         volatile uint32_t* abort_word, int32_t* err) {
-    const long long t0 = clock64();
-    for (;;) {
-        if (mbar_test(bar, parity)) return true;
-        if (*abort_word) return false;
-        if (clock64() - t0 > kWaitCycles) break;
-    }
-    *abort_word = 1u;
-    flag(err, PKV_DEVERR_WAIT_TIMEOUT);
-    return false;
-}
-
-// Wait for completion, ignoring the abort word (draining copies and MMAs).
-__device__ __forceinline__ void quiet_wait(uint32_t bar, uint32_t parity) {
-    const long long t0 = clock64();
-    while (!mbar_test(bar, parity) && clock64() - t0 <= kWaitCycles) {
-    }
 }
 
 // Diagnostic (pkv_selftest_wait_timeout, which = 2): one warp waits with the
@@ -672,6 +627,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
 // ------------------------------------------------------------------ host side
 
+}  // namespace
+
 // Q [num_tokens][num_heads][D] as 4-D: x = 64 columns, y = head, z = token,
 // w = 64-column half.  A box of 64 x g x (128 / g) x D/64 lands as [half][token]
 // [head][128 B] = [half][row][128 B], 128B-swizzled: the A operand of Q K^T.
@@ -713,6 +670,8 @@ pkv_status encode_block_map(CUtensorMap* tm, const void* pool, const pkv_cache_d
     if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (pool)");
     return PKV_OK;
 }
+
+namespace {
 
 template <typename T, int D, int BS>
 struct PrefillTag {};
