@@ -16,13 +16,18 @@ namespace {
 
 constexpr int kCopyThreads = 256;
 
-// One thread per 16-byte chunk of one (token, kv head) row, for K and V alike.
-// Consecutive threads cover consecutive chunks, so both the reads of `key` and
-// the writes into the pool are fully coalesced 128-bit accesses.
+// One warp per token (grid-stride over the tokens).  A token's keys are
+// num_kv_heads x head_dim contiguous elements of `key` (likewise `value`):
+// lane l reads 16-byte chunks l, l + 32, ... of both -- kAppendBatch of each in
+// flight before any store -- and writes each chunk into its (block, kv head)
+// row of the pool at the slot's offset.  Reads are fully coalesced; every
+// 256-byte (D = 128) or 128-byte (D = 64) row lands as whole 16-byte stores.
+constexpr int kAppendBatch = 4;
+
 __global__ void __launch_bounds__(kCopyThreads)
 append_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
               const uint4* __restrict__ key, const uint4* __restrict__ value,
-              const int64_t* __restrict__ slot_mapping, int64_t total_chunks,
+              const int64_t* __restrict__ slot_mapping, int64_t num_tokens,
               int32_t chunks_per_row, int32_t num_kv_heads, int32_t block_size,
               int64_t num_slots, int32_t* err_flag) {
     // let a decode launched behind this kernel start its set-up now; this kernel
@@ -30,24 +35,43 @@ append_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
     // stream, so it waits for that work before touching memory
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_chunks;
-         i += stride) {
-        const int64_t row = i / chunks_per_row;  // token * num_kv_heads + head
-        const int32_t c = static_cast<int32_t>(i - row * chunks_per_row);
-        const int64_t token = row / num_kv_heads;
-        const int32_t head = static_cast<int32_t>(row - token * num_kv_heads);
-        const int64_t slot = __ldg(slot_mapping + token);
-        if (slot < 0) continue;  // padding token
-        if (slot >= num_slots) {
-            if (c == 0 && head == 0 && err_flag) atomicOr(err_flag, PKV_DEVERR_BAD_SLOT);
-            continue;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int per_token = chunks_per_row * num_kv_heads;
+    for (int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < num_tokens;
+         t += warps) {
+        const int64_t slot = __ldg(slot_mapping + t);
+        const uint4* ks = key + t * per_token;
+        const uint4* vs = value + t * per_token;
+        for (int c0 = 0; c0 < per_token; c0 += 32 * kAppendBatch) {
+            uint4 kr[kAppendBatch], vr[kAppendBatch];
+#pragma unroll
+            for (int j = 0; j < kAppendBatch; ++j) {
+                const int c = c0 + 32 * j + lane;
+                if (c < per_token) {
+                    kr[j] = __ldg(ks + c);
+                    vr[j] = __ldg(vs + c);
+                }
+            }
+            if (slot < 0) break;  // padding token
+            if (slot >= num_slots) {
+                if (lane == 0 && c0 == 0 && err_flag) atomicOr(err_flag, PKV_DEVERR_BAD_SLOT);
+                break;
+            }
+            const int64_t block = slot / block_size;
+            const int64_t offset = slot - block * block_size;
+#pragma unroll
+            for (int j = 0; j < kAppendBatch; ++j) {
+                const int c = c0 + 32 * j + lane;
+                if (c < per_token) {
+                    const int head = c / chunks_per_row;
+                    const int cc = c - head * chunks_per_row;
+                    const int64_t dst = ((block * num_kv_heads + head) * block_size + offset) * chunks_per_row + cc;
+                    k_cache[dst] = kr[j];
+                    v_cache[dst] = vr[j];
+                }
+            }
         }
-        const int64_t block = slot / block_size;
-        const int64_t offset = slot - block * block_size;
-        const int64_t dst = ((block * num_kv_heads + head) * block_size + offset) * chunks_per_row + c;
-        k_cache[dst] = __ldg(key + i);
-        v_cache[dst] = __ldg(value + i);
     }
 }
 
@@ -143,9 +167,9 @@ extern "C" pkv_status paged_kv_append(const pkv_cache_desc* desc, void* k_cache,
     if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(key) || !aligned16(value))
         return fail(PKV_ERR_INVALID_ARG, "paged_kv_append: pools, key and value must be 16-byte aligned");
     const int32_t chunks_per_row = desc->head_dim * 2 / 16;
-    const int64_t total = static_cast<int64_t>(num_tokens) * desc->num_kv_heads * chunks_per_row;
-    const int64_t want = (total + kCopyThreads - 1) / kCopyThreads;
-    const int grid = static_cast<int>(want < 148 * 16 ? want : 148 * 16);
+    // one warp per token, at most a full device of warps (148 SMs x 8 CTAs)
+    const int64_t want = (static_cast<int64_t>(num_tokens) + kCopyThreads / 32 - 1) / (kCopyThreads / 32);
+    const int grid = static_cast<int>(want < 148 * 8 ? want : 148 * 8);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kCopyThreads);
@@ -157,8 +181,8 @@ extern "C" pkv_status paged_kv_append(const pkv_cache_desc* desc, void* k_cache,
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(
         &cfg, append_kernel, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
-        static_cast<const uint4*>(key), static_cast<const uint4*>(value), slot_mapping, total,
-        chunks_per_row, desc->num_kv_heads, desc->block_size,
+        static_cast<const uint4*>(key), static_cast<const uint4*>(value), slot_mapping,
+        static_cast<int64_t>(num_tokens), chunks_per_row, desc->num_kv_heads, desc->block_size,
         static_cast<int64_t>(desc->num_blocks) * desc->block_size, err_flag);
     note_launches(1);
     if (e == cudaSuccess) e = cudaGetLastError();
