@@ -142,11 +142,12 @@ __global__ void __launch_bounds__(kCaThreads, 1)
         tmem_alloc(sb + Lay::kMisc, kCaTmemCols);
         tmem_relinquish();
     }
-    // Launched as a programmatic dependent of the previous work in the stream:
-    // nothing global is read before it is done.  The balanced decode launched
-    // behind this kernel may start its set-up now; it waits for this grid to
-    // complete before it reads anything this kernel writes.
-    pdl_wait_primary();
+    // Launched behind the call's decode of the sequences' own tokens, as a
+    // programmatic dependent: it starts once every CTA before it has passed its
+    // own wait for the call's inputs, and reads only those inputs (queries, the
+    // pools, the tables) and writes only its own partials, so it runs without
+    // waiting; it waits for the kernels before it at the end, so the kernel
+    // behind it (launched early here) sees everything complete.
     pdl_launch_dependents();
     tc_fence_before();
     __syncthreads();
@@ -328,6 +329,7 @@ __global__ void __launch_bounds__(kCaThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kCaTmemCols);
     }
+    pdl_wait_primary();
 }
 
 template <typename T, int D, int BS>
@@ -389,20 +391,24 @@ pkv_status plan_groups(const pkv_cache_desc* desc, int32_t num_seqs, int32_t num
     }
     cg->start[num_groups] = num_groups > 0 ? group_start[num_groups] : 0;
     cg->tiles_per_item = items1 * desc->num_kv_heads >= kPrefixTwoTilesFrom ? 2 : 1;
-    int64_t base = 0, items = 0;
+    int64_t base = 0, items = 0, seqs = 0;
     for (int i = 0; i < num_groups; ++i) {
         const int n = cg->start[i + 1] - cg->start[i];
         const int64_t tiles = (cg->shared_tokens[i] + kPrefixKv - 1) / kPrefixKv;
         cg->chunks[i] = static_cast<int32_t>((tiles + cg->tiles_per_item - 1) / cg->tiles_per_item);
         cg->pre_base[i] = static_cast<int32_t>(base);
         cg->item_base[i] = static_cast<int32_t>(items);
+        cg->seq_base[i] = static_cast<int32_t>(seqs);
         base += static_cast<int64_t>(n) * num_heads * cg->chunks[i];
         items += static_cast<int64_t>(cg->chunks[i]) * ((n + seqs_per_tile - 1) / seqs_per_tile);
+        if (cg->shared_tokens[i] > 0) seqs += n;
         if (base > INT32_MAX || items > INT32_MAX)
             return fail(PKV_ERR_UNSUPPORTED, "shared-prefix decode: too many prefix partials");
     }
     cg->item_base[num_groups] = static_cast<int32_t>(items);
-    *slots = base;
+    cg->seq_base[num_groups] = static_cast<int32_t>(seqs);
+    cg->grouped_seqs = static_cast<int32_t>(seqs);
+    *slots = base + seqs * num_heads;
     return PKV_OK;
 }
 

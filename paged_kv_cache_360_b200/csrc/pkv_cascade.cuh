@@ -24,20 +24,30 @@ constexpr int kPrefixKv = 128;    // kv tokens of one prefix kv tile
 struct CascadeGroups {
     int32_t num_groups;
     int32_t tiles_per_item;                 // kv tiles of one prefix work item (1 or 2)
+    int32_t grouped_seqs;                   // sequences of the groups that share blocks
     int32_t start[kMaxGroups + 1];          // group i = sequences start[i] .. start[i+1]-1
     int32_t shared_tokens[kMaxGroups];      // tokens of the shared blocks (a multiple of bs)
     int32_t chunks[kMaxGroups];             // prefix partials per (sequence, head)
-    int32_t pre_base[kMaxGroups];           // first partial slot of the group
+    int32_t pre_base[kMaxGroups];           // first prefix partial slot of the group
+    int32_t seq_base[kMaxGroups + 1];       // grouped sequences before group i (sharing groups)
     int32_t item_base[kMaxGroups + 1];      // prefix work items before group i
-    float* pre_o;                           // [slot][D]   un-normalised partial O
-    float* pre_ml;                          // [slot][2]   partial (m, l), m in base-2 units
+    float* pre_o;                           // [slot][D]   un-normalised prefix partial O
+    float* pre_ml;                          // [slot][2]   prefix partial (m, l), m in base-2 units
+    float* own_o;                           // [grouped row][D]  the same over each sequence's own
+    float* own_ml;                          // [grouped row][2]  tokens (rows: sequence x head)
 };
 
-// Partial slot of (sequence b of group i, query head h, chunk c).
+// Prefix partial slot of (sequence b of group i, query head h, chunk c).
 __host__ __device__ __forceinline__ int64_t prefix_slot(const CascadeGroups& cg, int i, int b,
                                                          int num_heads, int h, int c) {
     return static_cast<int64_t>(cg.pre_base[i]) +
            (static_cast<int64_t>(b - cg.start[i]) * num_heads + h) * cg.chunks[i] + c;
+}
+
+// Row of (sequence b of group i, query head h) in own_o / own_ml.
+__host__ __device__ __forceinline__ int64_t own_row(const CascadeGroups& cg, int i, int b,
+                                                    int num_heads, int h) {
+    return (static_cast<int64_t>(cg.seq_base[i]) + (b - cg.start[i])) * num_heads + h;
 }
 
 // Index of the group holding sequence b, or -1.
@@ -49,6 +59,12 @@ __device__ __forceinline__ int group_of(const CascadeGroups& cg, int b) {
         else hi = mid;
     }
     return lo < cg.num_groups && cg.start[lo] <= b ? lo : -1;
+}
+
+// Index of the group holding sequence b if that group shares blocks, else -1.
+__device__ __forceinline__ int sharing_group_of(const CascadeGroups& cg, int b) {
+    const int i = group_of(cg, b);
+    return i >= 0 && cg.shared_tokens[i] > 0 ? i : -1;
 }
 
 // Tokens at the start of sequence b that the prefix kernel attends (0 outside
@@ -68,13 +84,18 @@ constexpr int kPrefixTwoTilesFrom = 296;
 
 // Lay out the group table for these shapes from the caller's host arrays
 // (group_start [num_groups + 1], group_shared_blocks [num_groups]); *slots =
-// prefix partial slots.  Errors are recorded for pkv_last_error().
+// prefix partial slots + own-token rows (each D + 2 floats).  Errors are
+// recorded for pkv_last_error().
 pkv_status plan_groups(const pkv_cache_desc* desc, int32_t num_seqs, int32_t num_heads,
                        int32_t max_blocks_per_seq, const int32_t* group_start,
                        const int32_t* group_shared_blocks, int32_t num_groups, CascadeGroups* cg,
                        int64_t* slots);
 
-// The prefix kernel over every work item of `cg` (pkv_cascade.cu).
+// The prefix kernel over every work item of `cg` (pkv_cascade.cu).  It reads
+// only inputs of the call, so it does not wait for the kernels launched before
+// it in the call (it is launched behind them, when the call's inputs are
+// complete); it waits for them before it exits, so that the kernel behind it
+// sees all of their results.
 pkv_status launch_prefix(const pkv_cache_desc* desc, const void* q, const void* k_cache,
                          const void* v_cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
                          int32_t num_seqs, int32_t num_heads, float scale, const CascadeGroups& cg,

@@ -758,15 +758,10 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const int sb = smeta[0], shk = smeta[1];
             const bool complete = (flags & (kMetaBegins | kMetaEnds)) == (kMetaBegins | kMetaEnds);
             const int64_t pslot = static_cast<int64_t>(c) * 2 + ((flags & kSegFirstInCta) ? 0 : 1);
-            // The segment that starts a grouped sequence's own tokens also
-            // takes the prefix kernel's partials of its rows, after the warps'.
+            // A sequence of a group that shares blocks: its complete result over
+            // its own tokens is a partial too (the prefix is folded in later).
             int pgrp = -1;
-            if constexpr (CASCADE) {
-                if (flags & kMetaBegins) {
-                    pgrp = group_of(cg, sb);
-                    if (pgrp >= 0 && cg.shared_tokens[pgrp] == 0) pgrp = -1;
-                }
-            }
+            if constexpr (CASCADE) pgrp = sharing_group_of(cg, sb);
             // Row by row: the weights 2^(m_w - M) once per row, then four columns
             // per lane (M = max_w m_w; acc = sum_w 2^(m_w - M) o_w; den likewise).
             for (int r = 0; r < group; ++r) {
@@ -775,15 +770,6 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 for (int w = 0; w < kConsumerWarps; ++w) {
                     mw[w] = mm[w * group + r];
                     M = fmaxf(M, mw[w]);
-                }
-                int64_t pre0 = 0;
-                int nchunk = 0;
-                if constexpr (CASCADE) {
-                    if (pgrp >= 0) {
-                        nchunk = cg.chunks[pgrp];
-                        pre0 = prefix_slot(cg, pgrp, sb, a.num_heads, shk * group + r, 0);
-                        for (int k = 0; k < nchunk; ++k) M = fmaxf(M, cg.pre_ml[(pre0 + k) * 2]);
-                    }
                 }
                 float f[kConsumerWarps], den = 0.f;
 #pragma unroll
@@ -802,19 +788,13 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         acc.z += f[w] * o.z;
                         acc.w += f[w] * o.w;
                     }
-                    if constexpr (CASCADE) {
-                        for (int k = 0; k < nchunk; ++k) {
-                            const float2 ml_k = *reinterpret_cast<const float2*>(cg.pre_ml + (pre0 + k) * 2);
-                            const float fk = ml_k.x == -INFINITY ? 0.f : exp2_approx(ml_k.x - M);
-                            const float4 o = *reinterpret_cast<const float4*>(cg.pre_o + (pre0 + k) * D + d0);
-                            acc.x += fk * o.x;
-                            acc.y += fk * o.y;
-                            acc.z += fk * o.z;
-                            acc.w += fk * o.w;
-                            den += fk * ml_k.y;
+                    if (complete && pgrp >= 0) {
+                        if constexpr (CASCADE) {
+                            const int64_t row = own_row(cg, pgrp, sb, a.num_heads, shk * group + r);
+                            *reinterpret_cast<float4*>(cg.own_o + row * D + d0) = acc;
+                            if (lane == 0) *reinterpret_cast<float2*>(cg.own_ml + row * 2) = make_float2(M, den);
                         }
-                    }
-                    if (complete) {
+                    } else if (complete) {
                         const float inv = den > 0.f ? 1.f / den : 0.f;
                         float r0, r1;
                         uint2 packed;
@@ -1005,6 +985,8 @@ __global__ void __launch_bounds__(kReduceThreads)
         const int n = s_len[slot];
         if (n == 0) continue;
         const int b = s_meta[slot][0], hk = s_meta[slot][1];
+        int pgrp = -1;  // a sequence of a sharing group: the chain's result stays a partial
+        if constexpr (CASCADE) pgrp = sharing_group_of(cg, b);
         // (row, 4 columns) per thread: M = max m_p, out = sum 2^(m_p - M) o_p / sum 2^(m_p - M) l_p
         for (int item = tid; item < group * (D / 4); item += kReduceThreads) {
             const int r = item / (D / 4);
@@ -1060,6 +1042,14 @@ __global__ void __launch_bounds__(kReduceThreads)
                     den += f * a.ws_ml[(p * group + r) * 2 + 1];
                 }
             }
+            if constexpr (CASCADE) {
+                if (pgrp >= 0) {
+                    const int64_t row = own_row(cg, pgrp, b, a.num_heads, hk * group + r);
+                    *reinterpret_cast<float4*>(cg.own_o + row * D + d0) = acc;
+                    if (d0 == 0) *reinterpret_cast<float2*>(cg.own_ml + row * 2) = make_float2(M, den);
+                    continue;
+                }
+            }
             const float inv = den > 0.f ? 1.f / den : 0.f;
             float r0, r1;
             uint2 packed;
@@ -1071,39 +1061,118 @@ __global__ void __launch_bounds__(kReduceThreads)
     }
 
     // sequences with no tokens: zeros (context lengths <= 0 count as empty);
-    // with CASCADE, a grouped sequence whose tokens are all shared: its prefix
-    // partials, merged in chunk order
+    // with CASCADE the sequences of sharing groups are written by
+    // cascade_finalize_kernel instead
     int k = 0;
     for (int b = c; b < a.num_seqs; b += grid, ++k) {
         const bool empty = k < 4 ? empty_seq[k] : own_tokens(b) <= 0;
         if (!empty) continue;
+        if constexpr (CASCADE) {
+            if (sharing_group_of(cg, b) >= 0) continue;
+        }
         T* o = static_cast<T*>(a.out) + static_cast<int64_t>(b) * a.num_heads * D;
-        int pgrp = -1;
-        if constexpr (CASCADE) {
-            pgrp = group_of(cg, b);
-            if (pgrp >= 0 && (cg.shared_tokens[pgrp] == 0 || __ldg(a.context_lens + b) <= 0)) pgrp = -1;
+        for (int idx = tid; idx < a.num_heads * D; idx += kReduceThreads) o[idx] = Pack<T>::one(0.f);
+    }
+}
+
+// The last kernel of the shared-prefix decode: for every sequence of a sharing
+// group, the partials of its heads over the shared blocks (one per prefix
+// chunk, from prefix_kernel) and over its own tokens (from the kernels above;
+// none when all its tokens are shared) merge by log-sum-exp, prefix chunks in
+// order, then the own tokens:
+//   M = max m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
+// One warp per (grouped sequence, head): lane k holds chunk k's (m, l) (32 at
+// a time), so the maximum and the weights take shuffles, not round trips;
+// every lane then reads four columns of each chunk's O, eight chunks in
+// flight.  Launched as a programmatic dependent of the prefix kernel, whose
+// completion implies that of every kernel before it in the call.
+constexpr int kFinalThreads = 128;
+constexpr int kFinalChunks = 8;  // chunks' O rows in flight per lane
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kFinalThreads)
+    cascade_finalize_kernel(const BalancedArgs a, const __grid_constant__ CascadeGroups cg) {
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int64_t row_all = static_cast<int64_t>(blockIdx.x) * (kFinalThreads / 32) + (threadIdx.x >> 5);
+    if (row_all >= static_cast<int64_t>(cg.grouped_seqs) * a.num_heads) return;
+    const int j = static_cast<int>(row_all / a.num_heads);  // grouped sequence
+    const int h = static_cast<int>(row_all - static_cast<int64_t>(j) * a.num_heads);
+    int grp = 0;
+    while (grp + 1 < cg.num_groups && cg.seq_base[grp + 1] <= j) ++grp;
+    while (grp < cg.num_groups && cg.shared_tokens[grp] == 0) ++grp;  // (seq_base skips them)
+    const int b = cg.start[grp] + (j - cg.seq_base[grp]);
+    const int L = clamp_len(__ldg(a.context_lens + b), a.max_len);
+    const bool has_own = L > cg.shared_tokens[grp];
+    const int nchunk = cg.chunks[grp];
+    const int64_t p0 = prefix_slot(cg, grp, b, a.num_heads, h, 0);
+    const int64_t orow = own_row(cg, grp, b, a.num_heads, h);
+    const int d0 = lane * 4;
+    pdl_wait_primary();
+
+    float M = -INFINITY;
+    for (int k0 = 0; k0 < nchunk; k0 += 32)
+        if (k0 + lane < nchunk) M = fmaxf(M, cg.pre_ml[(p0 + k0 + lane) * 2]);
+    float2 own_ml = make_float2(-INFINITY, 0.f);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (has_own) {
+        own_ml = *reinterpret_cast<const float2*>(cg.own_ml + orow * 2);
+        M = fmaxf(M, own_ml.x);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float den = 0.f;
+    for (int k0 = 0; k0 < nchunk; k0 += 32) {
+        float f = 0.f, l = 0.f;
+        if (k0 + lane < nchunk) {
+            const float2 x = *reinterpret_cast<const float2*>(cg.pre_ml + (p0 + k0 + lane) * 2);
+            f = x.x == -INFINITY ? 0.f : exp2_approx(x.x - M);
+            l = x.y;
         }
-        if (pgrp < 0) {
-            for (int idx = tid; idx < a.num_heads * D; idx += kReduceThreads) o[idx] = Pack<T>::one(0.f);
-            continue;
-        }
-        if constexpr (CASCADE) {
-            const int nchunk = cg.chunks[pgrp];
-            for (int idx = tid; idx < a.num_heads * D; idx += kReduceThreads) {
-                const int h = idx / D, d = idx - h * D;
-                const int64_t p0 = prefix_slot(cg, pgrp, b, a.num_heads, h, 0);
-                float M = -INFINITY;
-                for (int q = 0; q < nchunk; ++q) M = fmaxf(M, cg.pre_ml[(p0 + q) * 2]);
-                float acc = 0.f, den = 0.f;
-                for (int q = 0; q < nchunk; ++q) {
-                    const float mq = cg.pre_ml[(p0 + q) * 2];
-                    const float f = mq == -INFINITY ? 0.f : exp2_approx(mq - M);
-                    acc += f * cg.pre_o[(p0 + q) * D + d];
-                    den += f * cg.pre_ml[(p0 + q) * 2 + 1];
+        float dl = f * l;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, off);
+        den += dl;
+        const int n = min(32, nchunk - k0);
+        for (int q0 = 0; q0 < n; q0 += kFinalChunks) {
+            float4 o[kFinalChunks];
+#pragma unroll
+            for (int q = 0; q < kFinalChunks; ++q)
+                if (q0 + q < n && d0 < D)
+                    o[q] = *reinterpret_cast<const float4*>(cg.pre_o + (p0 + k0 + q0 + q) * D + d0);
+#pragma unroll
+            for (int q = 0; q < kFinalChunks; ++q) {
+                if (q0 + q < n) {
+                    const float fq = __shfl_sync(0xffffffffu, f, q0 + q);
+                    if (d0 < D) {
+                        acc.x += fq * o[q].x;
+                        acc.y += fq * o[q].y;
+                        acc.z += fq * o[q].z;
+                        acc.w += fq * o[q].w;
+                    }
                 }
-                o[idx] = Pack<T>::one(den > 0.f ? acc / den : 0.f);
             }
         }
+    }
+    if (has_own && own_ml.x != -INFINITY) {
+        const float f = exp2_approx(own_ml.x - M);
+        if (d0 < D) {
+            const float4 o = *reinterpret_cast<const float4*>(cg.own_o + orow * D + d0);
+            acc.x += f * o.x;
+            acc.y += f * o.y;
+            acc.z += f * o.z;
+            acc.w += f * o.w;
+        }
+        den += f * own_ml.y;
+    }
+    if (d0 < D) {
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        float r0, r1;
+        uint2 packed;
+        packed.x = Pack<T>::two(acc.x * inv, acc.y * inv, r0, r1);
+        packed.y = Pack<T>::two(acc.z * inv, acc.w * inv, r0, r1);
+        const int64_t bh = static_cast<int64_t>(b) * a.num_heads + h;
+        *reinterpret_cast<uint2*>(static_cast<T*>(a.out) + bh * D + d0) = packed;
     }
 }
 
@@ -1465,6 +1534,14 @@ namespace {
 
 size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 
+template <typename T, int D>
+cudaError_t launch_finalize(const BalancedArgs& a, const CascadeGroups& cg, cudaStream_t stream) {
+    const int64_t rows = static_cast<int64_t>(cg.grouped_seqs) * a.num_heads;
+    const int64_t per = kFinalThreads / 32;
+    return launch_dependent(cascade_finalize_kernel<T, D>, dim3(static_cast<unsigned>((rows + per - 1) / per)),
+                            dim3(kFinalThreads), 0, stream, a, cg);
+}
+
 }  // namespace
 }  // namespace pkv
 
@@ -1509,13 +1586,16 @@ extern "C" pkv_status paged_attention_decode_shared_prefix(
         return paged_attention_decode(desc, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
                                       context_lens, num_seqs, num_heads, scale, 0, workspace,
                                       workspace_bytes, err_flag, stream);
+    // workspace: balanced partials | prefix partials (o, then m, l) | own-token
+    // partials of the grouped rows (o, then m, l)
+    const int64_t own_rows = static_cast<int64_t>(cg.grouped_seqs) * num_heads;
+    const int64_t pre_slots = slots - own_rows;
     cg.pre_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256(plain));
-    cg.pre_ml = cg.pre_o + slots * desc->head_dim;
+    cg.pre_ml = cg.pre_o + pre_slots * desc->head_dim;
+    cg.own_o = cg.pre_ml + pre_slots * 2;
+    cg.own_ml = cg.own_o + own_rows * desc->head_dim;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if ((st = launch_prefix(desc, q, k_cache, v_cache, block_tables, max_blocks_per_seq, num_seqs,
-                            num_heads, scale, cg, err_flag, s)) != PKV_OK)
-        return st;
     CUtensorMap tk, tv;
     if ((st = encode_pool_map(&tk, k_cache, desc, 16)) != PKV_OK) return st;
     if ((st = encode_pool_map(&tv, v_cache, desc, 16)) != PKV_OK) return st;
@@ -1536,7 +1616,20 @@ extern "C" pkv_status paged_attention_decode_shared_prefix(
     a.num_blocks = desc->num_blocks;
     a.max_len = max_blocks_per_seq * desc->block_size;
     a.scale_log2 = scale * kLog2e;
-    return dispatch<RunCascade>(desc, tk, tv, a, cg, grid, smem, s);
+    // 1-2: every sequence's own tokens (balanced decode + chain merge); 3: the
+    // shared blocks (prefix kernel, runs as SMs free up); 4: the merge of the two
+    if ((st = dispatch<RunCascade>(desc, tk, tv, a, cg, grid, smem, s)) != PKV_OK) return st;
+    if ((st = launch_prefix(desc, q, k_cache, v_cache, block_tables, max_blocks_per_seq, num_seqs,
+                            num_heads, scale, cg, err_flag, s)) != PKV_OK)
+        return st;
+    cudaError_t e = desc->head_dim == 128
+                        ? (desc->dtype == PKV_BF16 ? launch_finalize<__nv_bfloat16, 128>(a, cg, s)
+                                                   : launch_finalize<__half, 128>(a, cg, s))
+                        : (desc->dtype == PKV_BF16 ? launch_finalize<__nv_bfloat16, 64>(a, cg, s)
+                                                   : launch_finalize<__half, 64>(a, cg, s));
+    note_launches(1);
+    if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+    return PKV_OK;
 }
 
 // ------------------------------------------------ decode without allocation
