@@ -200,14 +200,16 @@ pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* out, const v
  * reference counts and copy on write; [glossary] prefix caching).  The result
  * is paged_attention_decode's (same definition, same precision rules); only
  * the schedule differs:
+ *   - the balanced decode attends every sequence to its own tokens (those past
+ *     the shared ones); for the sequences of a group it leaves its results as
+ *     un-normalised partials (m, l, O) in the workspace;
  *   - the decode queries of 128 / g sequences of a group times the g heads of
  *     one kv head form one 128-row tile that attends to the group's shared
  *     blocks on the tensor cores (tcgen05), so each shared K/V row is read once
  *     per tile instead of once per sequence; chunks of 128 or 256 shared tokens
- *     leave un-normalised partials (m, l, O) in the workspace;
- *   - the balanced decode attends every sequence to its own tokens (those past
- *     the shared ones) and folds the prefix partials of its rows into its
- *     log-sum-exp merge, in a fixed order (warps, then prefix chunks).
+ *     leave partials too;
+ *   - a last kernel merges each grouped row's partials by log-sum-exp in a
+ *     fixed order (prefix chunks, then the own tokens) and writes `out`.
  * The reduction order depends only on the shapes and the groups, so results
  * are bit-identical under any permutation of physical blocks; they differ from
  * paged_attention_decode's by rounding only.
@@ -228,6 +230,8 @@ pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* out, const v
  *   blocks (PKV_ERR_UNSUPPORTED otherwise).
  *   workspace            device, >= paged_attention_shared_prefix_workspace_bytes
  *                        (...) for the same arguments, 256-byte aligned.
+ * Launches four kernels on `stream` (each a programmatic dependent of the one
+ * before).
  * Other arguments, layouts and errors as paged_attention_decode (the schedule
  * is always the balanced one).  The host arrays are read during the call only.
  */
@@ -246,10 +250,12 @@ pkv_status paged_attention_decode_shared_prefix(const pkv_cache_desc* desc, void
 /*
  * Workspace bytes of paged_attention_decode_shared_prefix: the balanced
  * decode's workspace (paged_attention_workspace_bytes with partition_size 0)
- * rounded up to 256 bytes, then float partial outputs [S][head_dim] and
- * (m, l) pairs [S][2], S = sum over groups that share blocks of (sequences x
+ * rounded up to 256 bytes; then the prefix partials, float O [S][head_dim] and
+ * (m, l) [S][2], S = sum over groups that share blocks of (sequences x
  * num_heads x chunks), chunks = ceil(shared tokens / (128 x tiles per chunk)),
- * 1 or 2 tiles per chunk.  0 on invalid arguments.
+ * 1 or 2 tiles per chunk; then the own-token partials of the grouped rows,
+ * float O [R][head_dim] and (m, l) [R][2], R = (sequences of groups that share
+ * blocks) x num_heads.  0 on invalid arguments.
  */
 size_t paged_attention_shared_prefix_workspace_bytes(const pkv_cache_desc* desc, int32_t num_seqs,
                                                      int32_t num_heads, int32_t max_blocks_per_seq,

@@ -14,8 +14,8 @@
 // One CTA takes (group, row tile, kv head, chunk of 1 or 2 kv tiles of 128
 // tokens) and writes, for every row, the chunk's un-normalised partial
 //   m = max_t s_t (base 2),  l = sum_t 2^(s_t - m),  o = sum_t 2^(s_t - m) V_t
-// into the workspace; the balanced decode of the sequences' own tokens folds
-// these partials into its log-sum-exp merge (pkv_decode.cu).
+// into the workspace; cascade_finalize_kernel (pkv_decode.cu) merges these
+// with the partials of each sequence's own tokens by log-sum-exp.
 //   warp 4   producer: Q tile (4-D TMA box: x = 64 columns, y = head, z =
 //            sequence, w = half), then per kv tile one 3-D box per (block,
 //            half) of K and of V, the blocks taken from the group's first

@@ -4,10 +4,10 @@
 // "PagedAttention" ops page, At a glance and How it works: sequences that share
 // a prompt point their block tables at the same physical blocks.  A group is a
 // run of consecutive sequences of the batch whose first `shared_tokens /
-// block_size` table entries are the same blocks; the decode attends every
-// query of the group to those blocks in one tensor-core pass (prefix_kernel)
-// and each sequence's own tokens with the balanced decode, and folds the two
-// into one softmax by log-sum-exp.
+// block_size` table entries are the same blocks; the decode attends each
+// sequence's own tokens with the balanced decode, every query of the group to
+// the shared blocks in one tensor-core pass (prefix_kernel), and merges the
+// two into one softmax by log-sum-exp (cascade_finalize_kernel).
 #pragma once
 
 #include <cuda_runtime.h>

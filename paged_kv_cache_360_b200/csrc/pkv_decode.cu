@@ -470,10 +470,10 @@ struct Chunk {
     int phys;             // this lane's physical block
 };
 
-// With CASCADE, sequences of a shared-prefix group attend here only to their
-// own tokens (from the group's shared_tokens on; units count from there), and
-// the segment that starts a (b, hk) folds in the prefix kernel's partials of
-// those rows (CascadeGroups: written before this kernel starts).
+// With CASCADE, sequences of a group that shares blocks attend here only to
+// their own tokens (from the group's shared_tokens on; units count from
+// there), and their results stay un-normalised partials (CascadeGroups
+// own_o / own_ml) for cascade_finalize_kernel to merge with the prefix.
 template <bool CASCADE>
 using GroupsOf = typename std::conditional<CASCADE, CascadeGroups, NoGroups>::type;
 
