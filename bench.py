@@ -241,7 +241,7 @@ def decode_device_sha256() -> str:
     h = hashlib.sha256()
     src = open(os.path.join(csrc, "pkv_decode.cu"), "rb").read()
     h.update(src[:src.find(b"// ------------------------------------------------------------------ host side")])
-    for name in ("pkv_attend.cuh", "pkv_ptx.cuh"):
+    for name in ("pkv_attend.cuh", "pkv_ptx.cuh", "pkv_cascade.cuh"):
         h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()
 
@@ -254,7 +254,7 @@ def prefill_device_sha256() -> str:
     h = hashlib.sha256()
     src = open(os.path.join(csrc, "pkv_prefill.cu"), "rb").read()
     h.update(src[:src.find(b"// ------------------------------------------------------------------ host side")])
-    for name in ("pkv_tc.cuh", "pkv_ptx.cuh"):
+    for name in ("pkv_tc.cuh", "pkv_ptx.cuh", "pkv_wait.cuh"):
         h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()
 
