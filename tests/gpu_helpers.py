@@ -75,12 +75,16 @@ def oracle_decode(wl, seqs=None, k=None, v=None, tables=None, threads=1):
 PARITY_LOG = []
 
 
-def report_parity(what, mabs, mrel, n):
+def report_parity(what, mabs, mrel, n, used):
     """Record and print one comparison's largest errors (the GPU tests' parity
-    report); with PKV_PARITY_REPORT set, the run's records are also written
-    there as JSON lines at the end of the session."""
-    PARITY_LOG.append({"case": what, "max_abs": mabs, "max_rel": mrel, "elements": n})
-    print(f"parity {what}: max abs {mabs:.3e}, max rel {mrel:.3e} over {n} elements")
+    report): max abs, max rel (over |ref| > 1e-3) and the largest fraction of
+    the per-element bound ATOL + RTOL |ref| used.  With PKV_PARITY_REPORT set,
+    the run's records are also written there as JSON lines at the end of the
+    session."""
+    PARITY_LOG.append({"case": what, "max_abs": mabs, "max_rel": mrel, "tol_used": used,
+                       "elements": n})
+    print(f"parity {what}: max abs {mabs:.3e}, max rel {mrel:.3e}, {used:.2f} of the bound, "
+          f"over {n} elements")
 
 
 def compare(gpu_out, ref, seqs=None, what=""):
@@ -98,8 +102,9 @@ def compare(gpu_out, ref, seqs=None, what=""):
     rel = err / np.maximum(np.abs(ref), 1e-30)
     mabs = float(err.max()) if err.size else 0.0
     mrel = float(np.where(np.abs(ref) > 1e-3, rel, 0).max()) if err.size else 0.0
+    used = float((err / bound).max()) if err.size else 0.0
     if what:
-        report_parity(what, mabs, mrel, int(err.size))
+        report_parity(what, mabs, mrel, int(err.size), used)
     return mabs, mrel
 
 
