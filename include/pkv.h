@@ -251,11 +251,12 @@ pkv_status paged_attention_decode_shared_prefix(const pkv_cache_desc* desc, void
  * Workspace bytes of paged_attention_decode_shared_prefix: the balanced
  * decode's workspace (paged_attention_workspace_bytes with partition_size 0)
  * rounded up to 256 bytes; then the prefix partials, float O [S][head_dim] and
- * (m, l) [S][2], S = sum over groups that share blocks of (sequences x
- * num_heads x chunks), chunks = ceil(shared tokens / (128 x tiles per chunk)),
- * 1 or 2 tiles per chunk; then the own-token partials of the grouped rows,
- * float O [R][head_dim] and (m, l) [R][2], R = (sequences of groups that share
- * blocks) x num_heads.  0 on invalid arguments.
+ * (m, l) [S][2] in whole 128-row tiles, S = 128 x num_kv_heads x (sum over
+ * groups that share blocks of ceil(sequences / (128 / g)) x chunks), g =
+ * num_heads / num_kv_heads, chunks = ceil(shared tokens / (128 x tiles per
+ * chunk)), 1 or 2 tiles per chunk; then the own-token partials of the grouped
+ * rows, float O [R][head_dim] and (m, l) [R][2], R = (sequences of groups that
+ * share blocks) x num_heads.  0 on invalid arguments.
  */
 size_t paged_attention_shared_prefix_workspace_bytes(const pkv_cache_desc* desc, int32_t num_seqs,
                                                      int32_t num_heads, int32_t max_blocks_per_seq,

@@ -95,8 +95,8 @@ struct PrefixArgs {
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(kCaThreads, 1)
     prefix_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                  const __grid_constant__ CUtensorMap tv, const PrefixArgs a,
-                  const __grid_constant__ CascadeGroups cg) {
+                  const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tp,
+                  const PrefixArgs a, const __grid_constant__ CascadeGroups cg) {
     using Lay = CaLayout<D>;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     constexpr uint32_t kIdescS = f16_idesc(kBf16, kPrefixRows, kPrefixKv, false);
@@ -124,7 +124,6 @@ __global__ void __launch_bounds__(kCaThreads, 1)
     const int g = 1 << a.log2_group;
     const int seqs_per_tile = kPrefixRows >> a.log2_group;
     const int s0 = cg.start[grp] + rt * seqs_per_tile;  // first sequence of the row tile
-    const int s_end = cg.start[grp + 1];
     const int shared = cg.shared_tokens[grp];
     const int n_tiles = (shared + kPrefixKv - 1) / kPrefixKv;
     const int t0 = chunk * cg.tiles_per_item;
@@ -137,6 +136,7 @@ __global__ void __launch_bounds__(kCaThreads, 1)
         prefetch_tensormap(&tq);
         prefetch_tensormap(&tk);
         prefetch_tensormap(&tv);
+        prefetch_tensormap(&tp);
     }
     if (warp == kCaMma) {
         tmem_alloc(sb + Lay::kMisc, kCaTmemCols);
@@ -208,27 +208,40 @@ __global__ void __launch_bounds__(kCaThreads, 1)
             mbar_arrive(bar(kCbP + j));
         }
         if (ok) ok = warp_wait(bar(kCbO), 0, abort_word, a.err);
+        // The tile's partial, rows as they stand (rows of other sequences
+        // included: the tile's slots are its own).  O goes from tensor memory to
+        // shared memory -- the Q and K_0 buffers, no longer read -- as D/32 boxes
+        // of [128 rows][128 B], 16-byte chunk c of row r at c ^ (r & 7) (the
+        // TMA's 128B swizzle, so that the stores of 8 consecutive rows hit 8 bank
+        // groups), then one TMA tensor store per box writes the tile
+        // contiguously.  Every softmax warp reaches the barrier, failed or not;
+        // the stores go out only if no role raised the abort word.
+        const int64_t row0 = (static_cast<int64_t>(item) * a.num_kv_heads + hk) * kPrefixRows;
+        const uint32_t stage = sb + Lay::kQ;
         if (ok) {
             tc_fence_after();
-            const int seq = s0 + (r >> a.log2_group);
-            const int h = hk * g + (r & (g - 1));
-            const bool store = seq < s_end && seq < a.num_seqs;
-            const int64_t slot = store ? prefix_slot(cg, grp, seq, a.num_heads, h, chunk) : 0;
-            float* dst = cg.pre_o + slot * D;
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
                 tmem_ld32(lane_base + kColO + 32u * c, o);
                 tmem_wait_ld();
-                if (store) {
-                    float4* d4 = reinterpret_cast<float4*>(dst + 32 * c);
+                const uint32_t rowaddr = stage + c * (kPrefixRows * 128) + r * 128;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        d4[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                            __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
-                }
+                for (int i = 0; i < 8; ++i)
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                                     rowaddr + ((i ^ (r & 7)) << 4)),
+                                 "r"(o[4 * i]), "r"(o[4 * i + 1]), "r"(o[4 * i + 2]), "r"(o[4 * i + 3])
+                                 : "memory");
             }
-            if (store) *reinterpret_cast<float2*>(cg.pre_ml + slot * 2) = make_float2(m2, l);
+            fence_proxy_async_smem();
+            *reinterpret_cast<float2*>(cg.pre_ml + (row0 + r) * 2) = make_float2(m2, l);
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (threadIdx.x == 0 && *abort_word == 0u) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c)
+                tma_store_2d(&tp, stage + c * (kPrefixRows * 128), 32 * c, static_cast<int32_t>(row0));
+            bulk_commit_and_wait_all();
         }
     } else if (warp == kCaProducer) {
         // --------------------------------------------------------- producer
@@ -337,23 +350,42 @@ struct PrefixTag {};
 
 template <typename T, int D, int BS>
 cudaError_t launch_prefix_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const PrefixArgs& a, const CascadeGroups& cg, cudaStream_t stream) {
+                            const CUtensorMap& tp, const PrefixArgs& a, const CascadeGroups& cg,
+                            cudaStream_t stream) {
     auto* k = prefix_kernel<T, D, BS>;
     cudaError_t e = opt_in_smem<PrefixTag<T, D, BS>>(reinterpret_cast<const void*>(k));
     if (e != cudaSuccess) return e;
     const dim3 grid(static_cast<unsigned>(cg.item_base[cg.num_groups]),
                     static_cast<unsigned>(a.num_kv_heads));
-    return launch_dependent(k, grid, dim3(kCaThreads), CaLayout<D>::kAlloc, stream, tq, tk, tv, a, cg);
+    return launch_dependent(k, grid, dim3(kCaThreads), CaLayout<D>::kAlloc, stream, tq, tk, tv, tp, a,
+                            cg);
 }
 
 template <typename T>
 cudaError_t launch_prefix_dt(int D, int BS, const CUtensorMap& tq, const CUtensorMap& tk,
-                             const CUtensorMap& tv, const PrefixArgs& a, const CascadeGroups& cg,
-                             cudaStream_t stream) {
-    if (D == 128) return BS == 16 ? launch_prefix_t<T, 128, 16>(tq, tk, tv, a, cg, stream)
-                                  : launch_prefix_t<T, 128, 32>(tq, tk, tv, a, cg, stream);
-    return BS == 16 ? launch_prefix_t<T, 64, 16>(tq, tk, tv, a, cg, stream)
-                    : launch_prefix_t<T, 64, 32>(tq, tk, tv, a, cg, stream);
+                             const CUtensorMap& tv, const CUtensorMap& tp, const PrefixArgs& a,
+                             const CascadeGroups& cg, cudaStream_t stream) {
+    if (D == 128) return BS == 16 ? launch_prefix_t<T, 128, 16>(tq, tk, tv, tp, a, cg, stream)
+                                  : launch_prefix_t<T, 128, 32>(tq, tk, tv, tp, a, cg, stream);
+    return BS == 16 ? launch_prefix_t<T, 64, 16>(tq, tk, tv, tp, a, cg, stream)
+                    : launch_prefix_t<T, 64, 32>(tq, tk, tv, tp, a, cg, stream);
+}
+
+// The prefix partials' O as 2-D fp32 (x = head_dim columns, y = tile rows), a
+// box of 32 columns (128 B) x 128 rows, 128B swizzle: the layout the prefix
+// kernel stages its tiles in.
+pkv_status encode_partial_map(CUtensorMap* tm, float* pre_o, int64_t rows, int D) {
+    auto encode = tensor_map_encoder();
+    if (!encode) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 4};
+    cuuint32_t box[2] = {32, static_cast<cuuint32_t>(kPrefixRows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, pre_o, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (prefix partials)");
+    return PKV_OK;
 }
 
 }  // namespace
@@ -396,11 +428,10 @@ pkv_status plan_groups(const pkv_cache_desc* desc, int32_t num_seqs, int32_t num
         const int n = cg->start[i + 1] - cg->start[i];
         const int64_t tiles = (cg->shared_tokens[i] + kPrefixKv - 1) / kPrefixKv;
         cg->chunks[i] = static_cast<int32_t>((tiles + cg->tiles_per_item - 1) / cg->tiles_per_item);
-        cg->pre_base[i] = static_cast<int32_t>(base);
         cg->item_base[i] = static_cast<int32_t>(items);
         cg->seq_base[i] = static_cast<int32_t>(seqs);
-        base += static_cast<int64_t>(n) * num_heads * cg->chunks[i];
         items += static_cast<int64_t>(cg->chunks[i]) * ((n + seqs_per_tile - 1) / seqs_per_tile);
+        base = items * desc->num_kv_heads * kPrefixRows;
         if (cg->shared_tokens[i] > 0) seqs += n;
         if (base > INT32_MAX || items > INT32_MAX)
             return fail(PKV_ERR_UNSUPPORTED, "shared-prefix decode: too many prefix partials");
@@ -421,12 +452,14 @@ pkv_status launch_prefix(const pkv_cache_desc* desc, const void* q, const void* 
                          int32_t* err_flag, cudaStream_t stream) {
     if (cg.item_base[cg.num_groups] == 0) return PKV_OK;
     const int g = num_heads / desc->num_kv_heads;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, tp;
     pkv_status st;
     if ((st = encode_q_map(&tq, q, desc->dtype, num_seqs, num_heads, desc->head_dim, g)) != PKV_OK)
         return st;
     if ((st = encode_block_map(&tk, k_cache, desc)) != PKV_OK) return st;
     if ((st = encode_block_map(&tv, v_cache, desc)) != PKV_OK) return st;
+    const int64_t rows = static_cast<int64_t>(cg.item_base[cg.num_groups]) * desc->num_kv_heads * kPrefixRows;
+    if ((st = encode_partial_map(&tp, cg.pre_o, rows, desc->head_dim)) != PKV_OK) return st;
     PrefixArgs a;
     a.tables = block_tables;
     a.err = err_flag;
@@ -439,9 +472,9 @@ pkv_status launch_prefix(const pkv_cache_desc* desc, const void* q, const void* 
     a.sl2 = scale * 1.4426950408889634f;
     cudaError_t e = desc->dtype == PKV_BF16
                         ? launch_prefix_dt<__nv_bfloat16>(desc->head_dim, desc->block_size, tq, tk, tv,
-                                                          a, cg, stream)
-                        : launch_prefix_dt<__half>(desc->head_dim, desc->block_size, tq, tk, tv, a, cg,
-                                                   stream);
+                                                          tp, a, cg, stream)
+                        : launch_prefix_dt<__half>(desc->head_dim, desc->block_size, tq, tk, tv, tp, a,
+                                                   cg, stream);
     note_launches(1);
     if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
     return PKV_OK;

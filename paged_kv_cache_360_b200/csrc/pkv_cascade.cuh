@@ -28,20 +28,31 @@ struct CascadeGroups {
     int32_t start[kMaxGroups + 1];          // group i = sequences start[i] .. start[i+1]-1
     int32_t shared_tokens[kMaxGroups];      // tokens of the shared blocks (a multiple of bs)
     int32_t chunks[kMaxGroups];             // prefix partials per (sequence, head)
-    int32_t pre_base[kMaxGroups];           // first prefix partial slot of the group
     int32_t seq_base[kMaxGroups + 1];       // grouped sequences before group i (sharing groups)
     int32_t item_base[kMaxGroups + 1];      // prefix work items before group i
-    float* pre_o;                           // [slot][D]   un-normalised prefix partial O
-    float* pre_ml;                          // [slot][2]   prefix partial (m, l), m in base-2 units
+    float* pre_o;                           // [item][kv head][128 rows][D]  un-normalised prefix
+    float* pre_ml;                          // [item][kv head][128 rows][2]  partial O and (m, l),
+                                            //   m in base-2 units (a row = a prefix tile row)
     float* own_o;                           // [grouped row][D]  the same over each sequence's own
     float* own_ml;                          // [grouped row][2]  tokens (rows: sequence x head)
 };
 
-// Prefix partial slot of (sequence b of group i, query head h, chunk c).
-__host__ __device__ __forceinline__ int64_t prefix_slot(const CascadeGroups& cg, int i, int b,
-                                                         int num_heads, int h, int c) {
-    return static_cast<int64_t>(cg.pre_base[i]) +
-           (static_cast<int64_t>(b - cg.start[i]) * num_heads + h) * cg.chunks[i] + c;
+// Prefix partial row of (sequence b of group i, query head h, chunk c): the
+// row of the prefix tile (row tile, chunk, kv head) that holds that query.
+// Chunk c + 1 of the same query is prefix_chunk_stride rows further.
+__host__ __device__ __forceinline__ int64_t prefix_row(const CascadeGroups& cg, int i, int b,
+                                                        int log2_group, int num_kv_heads, int h,
+                                                        int c) {
+    const int spt = kPrefixRows >> log2_group;  // sequences per row tile
+    const int rt = (b - cg.start[i]) / spt;
+    const int hk = h >> log2_group;
+    const int r = (((b - cg.start[i]) - rt * spt) << log2_group) + (h - (hk << log2_group));
+    const int64_t item = cg.item_base[i] + static_cast<int64_t>(rt) * cg.chunks[i] + c;
+    return (item * num_kv_heads + hk) * kPrefixRows + r;
+}
+
+__host__ __device__ __forceinline__ int64_t prefix_chunk_stride(int num_kv_heads) {
+    return static_cast<int64_t>(num_kv_heads) * kPrefixRows;
 }
 
 // Row of (sequence b of group i, query head h) in own_o / own_ml.
@@ -91,7 +102,8 @@ pkv_status plan_groups(const pkv_cache_desc* desc, int32_t num_seqs, int32_t num
                        const int32_t* group_shared_blocks, int32_t num_groups, CascadeGroups* cg,
                        int64_t* slots);
 
-// The prefix kernel over every work item of `cg` (pkv_cascade.cu).  It reads
+// The prefix kernel over every work item of `cg` (pkv_cascade.cu); pre_o is
+// written through a TMA tensor map, so it must be 16-byte aligned.  It reads
 // only inputs of the call, so it does not wait for the kernels launched before
 // it in the call (it is launched behind them, when the call's inputs are
 // complete); it waits for them before it exits, so that the kernel behind it

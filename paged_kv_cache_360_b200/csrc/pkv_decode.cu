@@ -1105,14 +1105,16 @@ __global__ void __launch_bounds__(kFinalThreads)
     const int L = clamp_len(__ldg(a.context_lens + b), a.max_len);
     const bool has_own = L > cg.shared_tokens[grp];
     const int nchunk = cg.chunks[grp];
-    const int64_t p0 = prefix_slot(cg, grp, b, a.num_heads, h, 0);
+    const int log2g = __ffs(a.group) - 1;  // a power of two in sharing groups
+    const int64_t p0 = prefix_row(cg, grp, b, log2g, a.num_kv_heads, h, 0);
+    const int64_t pstride = prefix_chunk_stride(a.num_kv_heads);
     const int64_t orow = own_row(cg, grp, b, a.num_heads, h);
     const int d0 = lane * 4;
     pdl_wait_primary();
 
     float M = -INFINITY;
     for (int k0 = 0; k0 < nchunk; k0 += 32)
-        if (k0 + lane < nchunk) M = fmaxf(M, cg.pre_ml[(p0 + k0 + lane) * 2]);
+        if (k0 + lane < nchunk) M = fmaxf(M, cg.pre_ml[(p0 + (k0 + lane) * pstride) * 2]);
     float2 own_ml = make_float2(-INFINITY, 0.f);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (has_own) {
@@ -1125,7 +1127,7 @@ __global__ void __launch_bounds__(kFinalThreads)
     for (int k0 = 0; k0 < nchunk; k0 += 32) {
         float f = 0.f, l = 0.f;
         if (k0 + lane < nchunk) {
-            const float2 x = *reinterpret_cast<const float2*>(cg.pre_ml + (p0 + k0 + lane) * 2);
+            const float2 x = *reinterpret_cast<const float2*>(cg.pre_ml + (p0 + (k0 + lane) * pstride) * 2);
             f = x.x == -INFINITY ? 0.f : exp2_approx(x.x - M);
             l = x.y;
         }
@@ -1139,7 +1141,7 @@ __global__ void __launch_bounds__(kFinalThreads)
 #pragma unroll
             for (int q = 0; q < kFinalChunks; ++q)
                 if (q0 + q < n && d0 < D)
-                    o[q] = *reinterpret_cast<const float4*>(cg.pre_o + (p0 + k0 + q0 + q) * D + d0);
+                    o[q] = *reinterpret_cast<const float4*>(cg.pre_o + (p0 + (k0 + q0 + q) * pstride) * D + d0);
 #pragma unroll
             for (int q = 0; q < kFinalChunks; ++q) {
                 if (q0 + q < n) {

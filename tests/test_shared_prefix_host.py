@@ -88,12 +88,14 @@ def test_workspace_bytes_count_the_prefix_partials():
     gs = (ctypes.c_int32 * 3)(0, 5, 9)
     gb = (ctypes.c_int32 * 2)(9, 0)
     # 9 shared blocks of 16 tokens = 144 tokens = 2 kv tiles, 1 tile per item
-    # (few items): 2 chunks x 5 sequences x 8 heads partial slots of D + 2 floats
+    # (few items): 5 sequences x g = 4 heads fit one 128-row tile, so 2 items
+    # (chunks) x 2 kv heads tiles of 128 rows; then 5 sequences x 8 heads
+    # own-token rows; every row D + 2 floats
     got = lib.paged_attention_shared_prefix_workspace_bytes(ctypes.byref(d), 9, 8, 12, gs, gb, 2)
     if got == 0:
         pytest.skip("no CUDA device to size the balanced part of the workspace")
     plain = lib.paged_attention_workspace_bytes(ctypes.byref(d), 9, 8, 12, 0)
-    assert got == ((plain + 255) // 256) * 256 + 2 * 5 * 8 * (128 + 2) * 4
+    assert got == ((plain + 255) // 256) * 256 + (2 * 2 * 128 + 5 * 8) * (128 + 2) * 4
 
 
 FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: validation fails first
