@@ -138,7 +138,8 @@ pkv_status swap_blocks(const pkv_cache_desc* desc, void* k_cache, void* v_cache,
  *     float [G][2][group][head_dim], partial maxima and sums float
  *     [G][2][group][2], partial descriptors int32 [G][2][4].
  *   partition_size > 0 (fixed): 0 when partition_size >= max_blocks_per_seq *
- *     block_size (no split); else float partial outputs
+ *     block_size (no split); else the balanced workspace above rounded up to
+ *     256 bytes, then the partitions' float partial outputs
  *     [num_seqs][num_heads][P_max][head_dim], then maxima and sums
  *     [num_seqs][num_heads][P_max] each, P_max = ceil(max_blocks_per_seq *
  *     block_size / partition_size).
@@ -177,8 +178,14 @@ size_t paged_attention_workspace_bytes(const pkv_cache_desc* desc, int32_t num_s
  *                   (log-sum-exp, in CTA order).  Results then depend on the
  *                   device's SM count (not on timing).
  *                   > 0 = fixed partitions of partition_size tokens (a multiple
- *                   of block_size), merged by log-sum-exp in partition order;
- *                   >= max_blocks_per_seq * block_size means no split.
+ *                   of block_size): each partition's un-normalised partial is
+ *                   computed on the balanced schedule (its segments stop at
+ *                   partition boundaries; a partition split across CTAs is
+ *                   merged in CTA order), then each row's partitions are
+ *                   merged by log-sum-exp in partition order (three kernels);
+ *                   results depend on the SM count as above.  >=
+ *                   max_blocks_per_seq * block_size means no split: one CTA per
+ *                   (sequence, kv head), independent of the device.
  *   workspace       device, >= paged_attention_workspace_bytes(...), 16-byte
  *                   aligned; may be NULL when that size is 0.
  *   err_flag        device int32 or NULL (PKV_DEVERR_BAD_BLOCK_ID,

@@ -133,7 +133,7 @@ struct FixedLayout {
 // Three CTAs per SM (at most 128 registers a thread: 15 warps leave 4 per SM
 // sub-partition): a CTA's start-up -- table entries, then the first copies --
 // overlaps the other two CTAs' streaming.
-template <typename T, int D, int BS, bool SPLIT>
+template <typename T, int D, int BS>
 __global__ void __launch_bounds__(kThreads, 3)
 decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const DecodeArgs a) {
@@ -155,7 +155,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     // Launched as a programmatic dependent of the previous kernel in the stream
     // (e.g. the append): nothing global is touched before that kernel is done.
     pdl_wait_primary();
-    if (SPLIT) pdl_launch_dependents();
 
     const int max_len = a.max_blocks_per_seq * BS;
     const int raw_len = __ldg(a.context_lens + b);
@@ -163,7 +162,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     if (raw_len != L && threadIdx.x == 0 && part == 0 && hk == 0)
         flag(a.err_flag, PKV_DEVERR_BAD_CONTEXT_LEN);
     const int t_begin = part * a.partition_tokens;
-    if (SPLIT && t_begin >= L) return;  // this partition holds no tokens
     const int t_end = min(t_begin + a.partition_tokens, L);
     const int blk_begin = t_begin / BS;
     const int nblk = (t_end - t_begin + BS - 1) / BS;
@@ -261,16 +259,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         float M, acc, den;
         combine_warps<D>(mo, mm, ml, kConsumerWarps, group, r, d, M, acc, den);
         const int64_t bh = static_cast<int64_t>(b) * a.num_heads + static_cast<int64_t>(hk) * group + r;
-        if (SPLIT) {
-            const int64_t slot = bh * a.max_partitions + part;
-            a.ws_o[slot * D + d] = acc;
-            if (d == 0) {
-                a.ws_m[slot] = M;
-                a.ws_l[slot] = den;
-            }
-        } else {
-            static_cast<T*>(a.out)[bh * D + d] = Pack<T>::one(den > 0.f ? acc / den : 0.f);
-        }
+        static_cast<T*>(a.out)[bh * D + d] = Pack<T>::one(den > 0.f ? acc / den : 0.f);
     }
 }
 
@@ -377,11 +366,19 @@ struct BalancedArgs {
     int32_t num_blocks;
     int32_t max_len;  // max_blocks_per_seq * block_size
     float scale_log2;
+    // fixed partitions (part_units > 0): every partition of part_units units
+    // leaves its partial in [row][partition] slots for reduce_kernel
+    int32_t part_units;
+    int32_t max_partitions;
+    float* part_o;  // [B][H][P_max][D]
+    float* part_m;  // [B][H][P_max]
+    float* part_l;  // [B][H][P_max]
 };
 
 struct SegDesc {
     int32_t b, hk, first, n;  // CTA-local index of the first unit, unit count
     int32_t blk0, len, flags, beg;  // beg: first token the segment's units count from
+    int32_t part, pad[3];           // partition of the segment (fixed partitions)
 };
 
 // The balanced kernel streams 16-token units: a block of 32 tokens is two units
@@ -465,6 +462,8 @@ struct Chunk {
     int b, hk, u0, cnt;   // sequence, kv head, first unit within (b, hk), units
     int len, nu;          // the sequence's length and its units per kv head
     int beg;              // first token of unit 0 (after the shared prefix, if any)
+    int pbeg, pend;       // units [pbeg, pend) of (b, hk) form the chunk's partition
+                          // (the whole (b, hk) without fixed partitions)
     int seg_start;        // the chunk opens a segment of seg_len units
     int seg_len;
     int phys;             // this lane's physical block
@@ -634,10 +633,14 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             ch.len = len;
             ch.nu = nu;
             ch.beg = beg;
-            ch.cnt = min(32, min(nu - ub, n_units - walked));
+            // with fixed partitions a segment never crosses a partition boundary
+            const int pu = a.part_units;
+            ch.pbeg = pu > 0 ? ub - ub % pu : 0;
+            ch.pend = pu > 0 ? min(nu, ch.pbeg + pu) : nu;
+            ch.cnt = min(32, min(ch.pend - ub, n_units - walked));
             if (ch.cnt <= 0) return false;  // lengths changed under the kernel
-            ch.seg_start = ub == 0 || walked == 0;
-            ch.seg_len = min(nu - ub, n_units - walked);
+            ch.seg_start = ub == ch.pbeg || walked == 0;
+            ch.seg_len = min(ch.pend - ub, n_units - walked);
             // the entries are checked when they are used, so the loads stay in flight
             ch.phys = lane < ch.cnt
                           ? __ldg(a.block_tables + static_cast<int64_t>(b) * a.max_blocks_per_seq +
@@ -671,9 +674,10 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         d.blk0 = cur.u0;
                         d.len = cur.len;
                         d.beg = cur.beg;
-                        d.flags = (cur.u0 == 0 ? kMetaBegins : 0) |
-                                  (cur.u0 + cur.seg_len == cur.nu ? kMetaEnds : 0) |
+                        d.flags = (cur.u0 == cur.pbeg ? kMetaBegins : 0) |
+                                  (cur.u0 + cur.seg_len == cur.pend ? kMetaEnds : 0) |
                                   (i == 0 ? kSegFirstInCta : 0);
+                        d.part = a.part_units > 0 ? cur.pbeg / a.part_units : 0;
                         // the arrive releases the descriptor's stores to the consumers
                         mbar_arrive_expect_tx(seg_full + 8 * ks, lay.qslot_bytes);
                         const T* qsrc = static_cast<const T*>(a.q) +
@@ -755,7 +759,7 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const int* smeta = reinterpret_cast<const int*>(ml + kConsumerWarps * group);
             const int flags = smeta[2];
             if (flags & kSegEnd) break;
-            const int sb = smeta[0], shk = smeta[1];
+            const int sb = smeta[0], shk = smeta[1], spart = smeta[3];
             const bool complete = (flags & (kMetaBegins | kMetaEnds)) == (kMetaBegins | kMetaEnds);
             const int64_t pslot = static_cast<int64_t>(c) * 2 + ((flags & kSegFirstInCta) ? 0 : 1);
             // A sequence of a group that shares blocks: its complete result over
@@ -794,6 +798,15 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                             *reinterpret_cast<float4*>(cg.own_o + row * D + d0) = acc;
                             if (lane == 0) *reinterpret_cast<float2*>(cg.own_ml + row * 2) = make_float2(M, den);
                         }
+                    } else if (complete && a.part_units > 0) {
+                        // a whole partition: its partial goes to its slot
+                        const int64_t bh = static_cast<int64_t>(sb) * a.num_heads + static_cast<int64_t>(shk) * group + r;
+                        const int64_t slot = bh * a.max_partitions + spart;
+                        *reinterpret_cast<float4*>(a.part_o + slot * D + d0) = acc;
+                        if (lane == 0) {
+                            a.part_m[slot] = M;
+                            a.part_l[slot] = den;
+                        }
                     } else if (complete) {
                         const float inv = den > 0.f ? 1.f / den : 0.f;
                         float r0, r1;
@@ -816,6 +829,7 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 meta[0] = sb;
                 meta[1] = shk;
                 meta[2] = kMetaValid | (flags & (kMetaBegins | kMetaEnds));
+                meta[3] = spart;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(mslot_empty + 8 * ms);  // the slot may be refilled
@@ -826,7 +840,8 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     // -------------------------------------------------------------- consumers
     // Hand this warp's state of segment `seg` (or, with flags = kSegEnd, the end
     // of the range) to the merge warp through merge slot seg % 2.
-    auto publish = [&](int seg, const SoftmaxState<D>& state, int b_, int hk_, int flags_) -> bool {
+    auto publish = [&](int seg, const SoftmaxState<D>& state, int b_, int hk_, int flags_,
+                       int part_) -> bool {
         const int ms = seg % kMergeSlots;
         if (seg >= kMergeSlots &&
             !__all_sync(0xffffffffu,
@@ -841,6 +856,7 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             smeta[0] = b_;
             smeta[1] = hk_;
             smeta[2] = flags_;
+            smeta[3] = part_;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(mslot_full + 8 * ms);
@@ -857,7 +873,7 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         const SegDesc d = descs[ks];
         if (d.flags & kSegEnd) {
-            ok = publish(seg, st, 0, 0, kSegEnd);  // the merge warp stops here
+            ok = publish(seg, st, 0, 0, kSegEnd, 0);  // the merge warp stops here
             break;
         }
         load_q_fragments<T, D>(qa, reinterpret_cast<const T*>(smem + lay.q_off + ks * lay.qslot_bytes),
@@ -882,7 +898,7 @@ balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (!ok) break;
 
         finish_row_sums(st);
-        if (!publish(seg, st, d.b, d.hk, d.flags)) {
+        if (!publish(seg, st, d.b, d.hk, d.flags, d.part)) {
             ok = false;
             break;
         }
@@ -907,7 +923,7 @@ constexpr int kShortChain = 4;    // chains up to this long are merged from regi
 template <typename T, int D, bool CASCADE>
 __global__ void __launch_bounds__(kReduceThreads)
     balanced_reduce_kernel(const BalancedArgs a, const __grid_constant__ GroupsOf<CASCADE> cg) {
-    __shared__ int s_meta[2 + kChainWindow][3];  // own slots 0 and 1, then slot 0 of c+1 ..
+    __shared__ int s_meta[2 + kChainWindow][4];  // own slots 0 and 1, then slot 0 of c+1 ..
     __shared__ int s_len[2];
     const int c = blockIdx.x;
     const int grid = gridDim.x;
@@ -934,16 +950,18 @@ __global__ void __launch_bounds__(kReduceThreads)
     if (tid < 2 + kChainWindow) {
         const int cc = tid < 2 ? c : c + tid - 1;
         const int slot = tid == 1 ? 1 : 0;
-        int m0 = 0, m1 = 0, m2 = 0;
+        int m0 = 0, m1 = 0, m2 = 0, m3 = 0;
         if (cc < grid) {
             const int32_t* m = a.ws_meta + (static_cast<int64_t>(cc) * 2 + slot) * 4;
             m0 = m[0];
             m1 = m[1];
             m2 = m[2];
+            m3 = m[3];
         }
         s_meta[tid][0] = m0;
         s_meta[tid][1] = m1;
         s_meta[tid][2] = m2;
+        s_meta[tid][3] = m3;
     }
     __syncthreads();
     if (tid < 2) {
@@ -952,24 +970,26 @@ __global__ void __launch_bounds__(kReduceThreads)
         int len = 0;
         const int f = s_meta[tid][2];
         if ((f & kMetaValid) && (f & kMetaBegins)) {
-            const int b = s_meta[tid][0], hk = s_meta[tid][1];
+            const int b = s_meta[tid][0], hk = s_meta[tid][1], part = s_meta[tid][3];
             len = 1;
             for (int k = 1;; ++k) {
-                int nf, nb, nhk;
+                int nf, nb, nhk, npart;
                 if (k <= kChainWindow) {
                     nb = s_meta[k + 1][0];
                     nhk = s_meta[k + 1][1];
                     nf = s_meta[k + 1][2];
+                    npart = s_meta[k + 1][3];
                 } else if (c + k < grid) {
                     const int32_t* m = a.ws_meta + static_cast<int64_t>(c + k) * 8;
                     nb = m[0];
                     nhk = m[1];
                     nf = m[2];
+                    npart = m[3];
                 } else {
                     nf = 0;
-                    nb = nhk = -1;
+                    nb = nhk = npart = -1;
                 }
-                if (!(nf & kMetaValid) || nb != b || nhk != hk) {  // a CTA of the chain is missing
+                if (!(nf & kMetaValid) || nb != b || nhk != hk || npart != part) {  // a CTA of the chain is missing
                     flag(a.err_flag, PKV_DEVERR_WAIT_TIMEOUT);
                     break;
                 }
@@ -984,7 +1004,7 @@ __global__ void __launch_bounds__(kReduceThreads)
     for (int slot = 0; slot < 2; ++slot) {
         const int n = s_len[slot];
         if (n == 0) continue;
-        const int b = s_meta[slot][0], hk = s_meta[slot][1];
+        const int b = s_meta[slot][0], hk = s_meta[slot][1], part = s_meta[slot][3];
         int pgrp = -1;  // a sequence of a sharing group: the chain's result stays a partial
         if constexpr (CASCADE) pgrp = sharing_group_of(cg, b);
         // (row, 4 columns) per thread: M = max m_p, out = sum 2^(m_p - M) o_p / sum 2^(m_p - M) l_p
@@ -1050,6 +1070,16 @@ __global__ void __launch_bounds__(kReduceThreads)
                     continue;
                 }
             }
+            if (a.part_units > 0) {  // a partition's partial, to its slot
+                const int64_t bh = static_cast<int64_t>(b) * a.num_heads + static_cast<int64_t>(hk) * group + r;
+                const int64_t pslot = bh * a.max_partitions + part;
+                *reinterpret_cast<float4*>(a.part_o + pslot * D + d0) = acc;
+                if (d0 == 0) {
+                    a.part_m[pslot] = M;
+                    a.part_l[pslot] = den;
+                }
+                continue;
+            }
             const float inv = den > 0.f ? 1.f / den : 0.f;
             float r0, r1;
             uint2 packed;
@@ -1062,7 +1092,9 @@ __global__ void __launch_bounds__(kReduceThreads)
 
     // sequences with no tokens: zeros (context lengths <= 0 count as empty);
     // with CASCADE the sequences of sharing groups are written by
-    // cascade_finalize_kernel instead
+    // cascade_finalize_kernel instead, with fixed partitions every sequence by
+    // reduce_kernel
+    if (a.part_units > 0) return;
     int k = 0;
     for (int b = c; b < a.num_seqs; b += grid, ++k) {
         const bool empty = k < 4 ? empty_seq[k] : own_tokens(b) <= 0;
@@ -1204,51 +1236,46 @@ pkv_status encode_pool_map(CUtensorMap* tm, const void* pool, const pkv_cache_de
     return PKV_OK;
 }
 
-template <typename T, int D, int BS, bool SPLIT>
+template <typename T, int D, int BS>
 struct FixedTag {};
 template <typename T, int D, int BS, bool CASCADE>
 struct BalancedTag {};
 
+// One CTA per (sequence, kv head): the decode without a split.
 template <typename T, int D, int BS>
-pkv_status launch_fixed(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a,
-                        int32_t num_seqs, bool split, cudaStream_t stream) {
+pkv_status launch_unsplit(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a,
+                          int32_t num_seqs, cudaStream_t stream) {
     using Lay = FixedLayout<D, BS>;
-    const dim3 grid(static_cast<unsigned>(num_seqs) * a.num_kv_heads,
-                    split ? static_cast<unsigned>(a.max_partitions) : 1u);
-    cudaError_t e;
-    if (split) {
-        auto k = decode_kernel<T, D, BS, true>;
-        if ((e = opt_in_smem<FixedTag<T, D, BS, true>>(reinterpret_cast<const void*>(k))) != cudaSuccess)
-            return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
-        e = launch_dependent(k, grid, dim3(kThreads), Lay::kSmemBytes, stream, tk, tv, a);
-        note_launches(1);
-        if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
-        // The merge launches as a programmatic dependent of the partition
-        // kernel: its CTAs may start during the partition kernel's tail and wait
-        // in griddepcontrol.wait for the results.
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(num_seqs) * a.num_heads);
-        const bool wide = a.max_partitions >= kWideReduceFrom;
-        cfg.blockDim = dim3((wide ? 4 : 1) * D);
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        const int32_t max_len = a.max_blocks_per_seq * BS;
-        e = wide ? cudaLaunchKernelEx(&cfg, reduce_kernel<T, D, 4>, a, max_len)
-                 : cudaLaunchKernelEx(&cfg, reduce_kernel<T, D, 1>, a, max_len);
-        note_launches(1);
-        if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
-    } else {
-        auto k = decode_kernel<T, D, BS, false>;
-        if ((e = opt_in_smem<FixedTag<T, D, BS, false>>(reinterpret_cast<const void*>(k))) != cudaSuccess)
-            return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
-        e = launch_dependent(k, grid, dim3(kThreads), Lay::kSmemBytes, stream, tk, tv, a);
-        note_launches(1);
-        if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
-    }
+    auto k = decode_kernel<T, D, BS>;
+    cudaError_t e = opt_in_smem<FixedTag<T, D, BS>>(reinterpret_cast<const void*>(k));
+    if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+    e = launch_dependent(k, dim3(static_cast<unsigned>(num_seqs) * a.num_kv_heads), dim3(kThreads),
+                         Lay::kSmemBytes, stream, tk, tv, a);
+    note_launches(1);
+    if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
+    return PKV_OK;
+}
+
+// The merge of fixed partitions, behind the kernels that wrote them: one CTA of
+// D threads (four groups of D when rows have many partitions) per (sequence,
+// query head), a programmatic dependent that waits for their results.
+template <typename T, int D>
+pkv_status launch_partition_merge(const DecodeArgs& a, int32_t num_seqs, int32_t max_len,
+                                  cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(num_seqs) * a.num_heads);
+    const bool wide = a.max_partitions >= kWideReduceFrom;
+    cfg.blockDim = dim3((wide ? 4 : 1) * D);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, reduce_kernel<T, D, 4>, a, max_len)
+                         : cudaLaunchKernelEx(&cfg, reduce_kernel<T, D, 1>, a, max_len);
+    note_launches(1);
+    if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
     return PKV_OK;
 }
 
@@ -1334,10 +1361,16 @@ struct GridOf {
     static pkv_status run(int group, int* grid, int* smem) { return balanced_grid<T, D, BS>(group, grid, smem); }
 };
 template <typename T, int D, int BS>
-struct RunFixed {
+struct RunUnsplit {
     static pkv_status run(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a,
-                          int32_t num_seqs, bool split, cudaStream_t st) {
-        return launch_fixed<T, D, BS>(tk, tv, a, num_seqs, split, st);
+                          int32_t num_seqs, cudaStream_t st) {
+        return launch_unsplit<T, D, BS>(tk, tv, a, num_seqs, st);
+    }
+};
+template <typename T, int D, int BS>
+struct RunPartitionMerge {
+    static pkv_status run(const DecodeArgs& a, int32_t num_seqs, int32_t max_len, cudaStream_t st) {
+        return launch_partition_merge<T, D>(a, num_seqs, max_len, st);
     }
 };
 template <typename T, int D, int BS>
@@ -1355,9 +1388,9 @@ struct RunCascade {
     }
 };
 
-// Workspace of the fixed-partition path (0 when it does not split).
-size_t fixed_workspace(const pkv_cache_desc* d, int32_t num_seqs, int32_t num_heads,
-                       int32_t max_blocks_per_seq, int32_t P) {
+// Partition partials of the fixed-partition path (0 when it does not split).
+size_t partition_slots_bytes(const pkv_cache_desc* d, int32_t num_seqs, int32_t num_heads,
+                             int32_t max_blocks_per_seq, int32_t P) {
     const int64_t max_len = static_cast<int64_t>(max_blocks_per_seq) * d->block_size;
     if (P == 0 || P >= max_len) return 0;
     const int64_t pmax = (max_len + P - 1) / P;
@@ -1369,6 +1402,8 @@ size_t balanced_workspace(int grid, int group, int D) {
     return static_cast<size_t>(grid) * 2 *
            (static_cast<size_t>(group) * (D + 2) * sizeof(float) + 4 * sizeof(int32_t));
 }
+
+size_t round256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 
 }  // namespace
 }  // namespace pkv
@@ -1396,13 +1431,15 @@ extern "C" size_t paged_attention_workspace_bytes(const pkv_cache_desc* desc, in
     if (check_desc(desc) != PKV_OK || num_seqs <= 0 || num_heads <= 0 || max_blocks_per_seq <= 0 ||
         partition_size < 0 || num_heads % desc->num_kv_heads != 0)
         return 0;
-    if (partition_size > 0)
-        return fixed_workspace(desc, num_seqs, num_heads, max_blocks_per_seq, partition_size);
+    const size_t parts =
+        partition_slots_bytes(desc, num_seqs, num_heads, max_blocks_per_seq, partition_size);
+    if (partition_size > 0 && parts == 0) return 0;  // fixed partitions, no split
     const int group = num_heads / desc->num_kv_heads;
     if (group > 16) return 0;
     int grid = 0, smem = 0;
     if (dispatch<GridOf>(desc, group, &grid, &smem) != PKV_OK) return 0;
-    return balanced_workspace(grid, group, desc->head_dim);
+    const size_t balanced = balanced_workspace(grid, group, desc->head_dim);
+    return parts ? round256(balanced) + parts : balanced;
 }
 
 namespace pkv {
@@ -1507,26 +1544,60 @@ extern "C" pkv_status paged_attention_decode(const pkv_cache_desc* desc, void* o
     a.num_blocks = desc->num_blocks;
     a.scale_log2 = scale * kLog2e;
     if (split) {
+        // Fixed partitions on the balanced schedule: its segments stop at
+        // partition boundaries, every partition's partial lands in its slot
+        // (whole ones from the decode's merge warp, split ones from the chain
+        // merge), and reduce_kernel merges each row's partitions in order.
         const int64_t pmax = (max_len + partition_size - 1) / partition_size;
         if (pmax > 65535) return fail(PKV_ERR_UNSUPPORTED, "too many partitions (> 65535)");
-        const size_t need = fixed_workspace(desc, num_seqs, num_heads, max_blocks_per_seq, partition_size);
+        int grid = 0, smem = 0;
+        if ((st = dispatch<GridOf>(desc, static_cast<int>(group), &grid, &smem)) != PKV_OK) return st;
+        const size_t balanced = balanced_workspace(grid, group, desc->head_dim);
+        const size_t need = round256(balanced) +
+                            partition_slots_bytes(desc, num_seqs, num_heads, max_blocks_per_seq,
+                                                  partition_size);
         if (!workspace || workspace_bytes < need)
             return fail(PKV_ERR_WORKSPACE_TOO_SMALL, "paged_attention_decode: workspace too small");
         if (!aligned(workspace, 16))
             return fail(PKV_ERR_INVALID_ARG, "paged_attention_decode: workspace must be 16-byte aligned");
         const int64_t rows = static_cast<int64_t>(num_seqs) * num_heads * pmax;
-        a.ws_o = static_cast<float*>(workspace);
+        a.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(balanced));
         a.ws_m = a.ws_o + rows * desc->head_dim;
         a.ws_l = a.ws_m + rows;
         a.partition_tokens = partition_size;
         a.max_partitions = static_cast<int32_t>(pmax);
-    } else {
-        a.partition_tokens = static_cast<int32_t>(max_len);
-        a.max_partitions = 1;
+        BalancedArgs ba = {};
+        ba.out = out;
+        ba.q = q;
+        ba.block_tables = block_tables;
+        ba.context_lens = context_lens;
+        ba.ws_o = static_cast<float*>(workspace);
+        ba.ws_ml = ba.ws_o + static_cast<int64_t>(grid) * 2 * group * desc->head_dim;
+        ba.ws_meta = reinterpret_cast<int32_t*>(ba.ws_ml + static_cast<int64_t>(grid) * 2 * group * 2);
+        ba.err_flag = err_flag;
+        ba.num_seqs = num_seqs;
+        ba.num_heads = num_heads;
+        ba.num_kv_heads = desc->num_kv_heads;
+        ba.group = group;
+        ba.max_blocks_per_seq = max_blocks_per_seq;
+        ba.num_blocks = desc->num_blocks;
+        ba.max_len = static_cast<int32_t>(max_len);
+        ba.scale_log2 = scale * kLog2e;
+        ba.part_units = partition_size / 16;
+        ba.max_partitions = static_cast<int32_t>(pmax);
+        ba.part_o = a.ws_o;
+        ba.part_m = a.ws_m;
+        ba.part_l = a.ws_l;
+        if ((st = encode_pool_map(&tk, k_cache, desc, 16)) != PKV_OK) return st;
+        if ((st = encode_pool_map(&tv, v_cache, desc, 16)) != PKV_OK) return st;
+        if ((st = dispatch<RunBalanced>(desc, tk, tv, ba, grid, smem, s)) != PKV_OK) return st;
+        return dispatch<RunPartitionMerge>(desc, a, num_seqs, static_cast<int32_t>(max_len), s);
     }
+    a.partition_tokens = static_cast<int32_t>(max_len);
+    a.max_partitions = 1;
     if ((st = encode_pool_map(&tk, k_cache, desc, desc->block_size)) != PKV_OK) return st;
     if ((st = encode_pool_map(&tv, v_cache, desc, desc->block_size)) != PKV_OK) return st;
-    return dispatch<RunFixed>(desc, tk, tv, a, num_seqs, split, s);
+    return dispatch<RunUnsplit>(desc, tk, tv, a, num_seqs, s);
 }
 
 // ------------------------------------------------------ shared-prefix decode
