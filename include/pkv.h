@@ -143,7 +143,8 @@ pkv_status swap_blocks(const pkv_cache_desc* desc, void* k_cache, void* v_cache,
  *     [num_seqs][num_heads][P_max][head_dim], then maxima and sums
  *     [num_seqs][num_heads][P_max] each, P_max = ceil(max_blocks_per_seq *
  *     block_size / partition_size).
- * Returns 0 on invalid arguments.
+ * Returns 0 on invalid arguments, and when a split is asked for but no CUDA
+ * device is visible (the balanced part is sized by the current device).
  */
 size_t paged_attention_workspace_bytes(const pkv_cache_desc* desc, int32_t num_seqs,
                                        int32_t num_heads, int32_t max_blocks_per_seq,
