@@ -577,15 +577,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 for (int j = 0; ok && j < nkv; ++j) {
                     const uint32_t vs =
                         sb + Lay::kStage0 + 2u * (j % kPfStages) * Lay::kTile + Lay::kTile;
-                    bool v_ready = false, k_ready = false;
+                    // V(j) and K(j + 1) first: they have usually landed by now.  A
+                    // barrier check issues nothing for ~100 cycles even on a
+                    // completed phase, and between the MMA groups below it would
+                    // sit on the softmax -> P V -> S path with the tensor pipe idle.
+                    if (!(ok = one_wait(bar(kBarVFull + j % kPfStages), (j / kPfStages) & 1, abort_word,
+                                        a.err)))
+                        break;
+                    if (j + 1 < nkv && !(ok = one_wait(bar(kBarKFull + (j + 1) % kPfStages),
+                                                        ((j + 1) / kPfStages) & 1, abort_word, a.err)))
+                        break;
                     for (int t = 0; ok && t < 2; ++t) {
                         const int nkv_of_t = t ? nkv1 : nkv0;
                         if (j >= nkv_of_t) continue;
                         if (!(ok = one_wait(bar(kBarPFull + t), j & 1, abort_word, a.err))) break;
-                        if (!v_ready && !(ok = one_wait(bar(kBarVFull + j % kPfStages),
-                                                         (j / kPfStages) & 1, abort_word, a.err)))
-                            break;
-                        v_ready = true;
                         tc_fence_after();
                         // P V: P in S_t's columns 0-63 (and, in the first kv
                         // tile, its rounding residual in columns 64-127)
@@ -597,15 +602,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                                            sw128_desc(vs + k * 16 * 128, Lay::kHalfBytes, 1024), kIdescO,
                                            (j > 0 || part > 0 || k > 0) ? 1u : 0u);
                         if (j + 1 == nkv_of_t) mma_commit(bar(kBarODone + t));
-                        if (j + 1 < nkv_of_t) {
-                            if (!k_ready && !(ok = one_wait(bar(kBarKFull + (j + 1) % kPfStages),
-                                                            ((j + 1) / kPfStages) & 1, abort_word,
-                                                            a.err)))
-                                break;
-                            k_ready = true;
-                            tc_fence_after();
-                            issue_s(t, j + 1);
-                        }
+                        if (j + 1 < nkv_of_t) issue_s(t, j + 1);
                     }
                     if (!ok) break;
                     mma_commit(bar(kBarVEmpty + j % kPfStages));
