@@ -28,7 +28,8 @@
 //               than 2^8.  The MMAs of one thread complete in issue order, so
 //               when S_t(j) is complete so is P_t V(j-1): O_t is stable during
 //               the softmax and needs no extra wait.  At the end, O / l goes to
-//               global memory.
+//               global memory: a full tile as one bulk tensor store staged in
+//               its (by then free) Q buffer, a partial tile row by row.
 //
 // Every mbarrier wait is bounded and warp-uniform; a timeout raises a shared
 // abort word, records PKV_DEVERR_WAIT_TIMEOUT and every role drains its
@@ -222,7 +223,8 @@ __device__ void find_item(const PrefillArgs& a, int cap, int tok_per_tile, int i
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                   const __grid_constant__ CUtensorMap tv, const PrefillArgs a) {
+                   const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
+                   const PrefillArgs a) {
     using Lay = PfLayout<D>;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     constexpr uint32_t kIdescS = f16_idesc(kBf16, kPfRows, kPfKv, false);
@@ -259,6 +261,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         prefetch_tensormap(&tq);
         prefetch_tensormap(&tk);
         prefetch_tensormap(&tv);
+        prefetch_tensormap(&to);
     }
     if (warp == kMmaWarp) {
         tmem_alloc(sb + Lay::kMisc, kTmemCols);
@@ -448,12 +451,54 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 mbar_arrive(bar(kBarPFull + t));
             }
             if (ok && my_nkv > 0) ok = warp_wait(bar(kBarODone + t), 0, abort_word, a.err);
-            if (ok && my_nkv > 0) {
+            // A full tile (every row a query of this sequence) goes out as one
+            // bulk tensor store of the tile's rows, staged in its Q buffer (free
+            // once the tile's last Q K^T, which completes before its last P V,
+            // is done); other tiles store row by row.  Tile-uniform choice, so
+            // the tile's four warps all meet the named barrier below.
+            const bool full = my_nkv > 0 && hi_t - lo_t == tok_per_tile && q0 + lo_t >= 0 &&
+                              static_cast<int64_t>(q0) + lo_t + tok_per_tile <= a.num_tokens;
+            const int64_t qrow = static_cast<int64_t>(q0) + lo_t + tok;
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            if (full) {
+                const uint32_t q_t = sb + Lay::kQ + t * Lay::kTile;
+                if (ok) {
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(o_addr + c * 32, o);
+                        tmem_wait_ld();
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float r0, r1;
+                            pk[i] = Pack<T>::two(__uint_as_float(o[2 * i]) * inv,
+                                                 __uint_as_float(o[2 * i + 1]) * inv, r0, r1);
+                        }
+                        // columns 32 c .. 32 c + 31: half c / 2, 16-byte chunks
+                        // 4 (c % 2) .. + 3 of the row, 128B-swizzled like the TMA's
+                        const uint32_t row = q_t + (c >> 1) * Lay::kHalfBytes + r * 128u;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint32_t chunk = (static_cast<uint32_t>((c & 1) * 4 + i) ^ (r & 7u)) * 16u;
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + chunk),
+                                         "r"(pk[4 * i]), "r"(pk[4 * i + 1]), "r"(pk[4 * i + 2]),
+                                         "r"(pk[4 * i + 3])
+                                         : "memory");
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                asm volatile("bar.sync %0, 128;" ::"r"(1 + t) : "memory");
+                if (r == 0 && ok && *abort_word == 0u) {
+                    tma_store_4d(&to, q_t, 0, hk * g, q0 + lo_t, 0);
+                    bulk_commit_and_wait_read();
+                }
+            } else if (ok && my_nkv > 0) {
                 tc_fence_after();
-                const int64_t qrow = static_cast<int64_t>(q0) + lo_t + tok;
                 const bool store = valid && qrow >= 0 && qrow < a.num_tokens;
                 if (valid && !store) flag(a.err, PKV_DEVERR_BAD_QUERY_COUNT);
-                const float inv = l > 0.f ? 1.f / l : 0.f;
                 T* dst = static_cast<T*>(a.out) +
                          (qrow * a.num_heads + static_cast<int64_t>(hk) * g + jh) * D;
 #pragma unroll 1
@@ -675,6 +720,7 @@ struct PrefillTag {};
 
 template <typename T, int D, int BS>
 cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const CUtensorMap& to,
                            const PrefillArgs& a, cudaStream_t stream) {
     auto* k = prefill_kernel<T, D, BS>;
     cudaError_t e = opt_in_smem<PrefillTag<T, D, BS>>(reinterpret_cast<const void*>(k));
@@ -683,16 +729,17 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
     const int tok_per_tile = kPfRows >> a.log2_group;
     dim3 grid(static_cast<unsigned>(a.num_tokens / (2 * tok_per_tile) + a.num_seqs),
               static_cast<unsigned>(a.num_kv_heads));
-    return launch_dependent(k, grid, dim3(kPfThreads), PfLayout<D>::kAlloc, stream, tq, tk, tv, a);
+    return launch_dependent(k, grid, dim3(kPfThreads), PfLayout<D>::kAlloc, stream, tq, tk, tv, to, a);
 }
 
 template <typename T>
 cudaError_t launch_prefill_dt(int D, int BS, const CUtensorMap& tq, const CUtensorMap& tk,
-                              const CUtensorMap& tv, const PrefillArgs& a, cudaStream_t stream) {
-    if (D == 128) return BS == 16 ? launch_prefill<T, 128, 16>(tq, tk, tv, a, stream)
-                                  : launch_prefill<T, 128, 32>(tq, tk, tv, a, stream);
-    return BS == 16 ? launch_prefill<T, 64, 16>(tq, tk, tv, a, stream)
-                    : launch_prefill<T, 64, 32>(tq, tk, tv, a, stream);
+                              const CUtensorMap& tv, const CUtensorMap& to, const PrefillArgs& a,
+                              cudaStream_t stream) {
+    if (D == 128) return BS == 16 ? launch_prefill<T, 128, 16>(tq, tk, tv, to, a, stream)
+                                  : launch_prefill<T, 128, 32>(tq, tk, tv, to, a, stream);
+    return BS == 16 ? launch_prefill<T, 64, 16>(tq, tk, tv, to, a, stream)
+                    : launch_prefill<T, 64, 32>(tq, tk, tv, to, a, stream);
 }
 
 }  // namespace
@@ -736,8 +783,11 @@ extern "C" pkv_status paged_attention_prefill(const pkv_cache_desc* desc, void* 
     if (static_cast<int64_t>(num_tokens) / (kPfRows / g) + num_seqs > INT32_MAX)
         return fail(PKV_ERR_UNSUPPORTED, "too many query tiles");
 
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if ((st = encode_q_map(&tq, q, desc->dtype, num_tokens, num_heads, desc->head_dim, g)) != PKV_OK)
+        return st;
+    // out has q's shape: the same map describes a tile of output rows
+    if ((st = encode_q_map(&to, out, desc->dtype, num_tokens, num_heads, desc->head_dim, g)) != PKV_OK)
         return st;
     if ((st = encode_block_map(&tk, k_cache, desc)) != PKV_OK) return st;
     if ((st = encode_block_map(&tv, v_cache, desc)) != PKV_OK) return st;
@@ -760,8 +810,9 @@ extern "C" pkv_status paged_attention_prefill(const pkv_cache_desc* desc, void* 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = desc->dtype == PKV_BF16
                         ? launch_prefill_dt<__nv_bfloat16>(desc->head_dim, desc->block_size, tq, tk,
-                                                           tv, a, s)
-                        : launch_prefill_dt<__half>(desc->head_dim, desc->block_size, tq, tk, tv, a, s);
+                                                           tv, to, a, s)
+                        : launch_prefill_dt<__half>(desc->head_dim, desc->block_size, tq, tk, tv, to, a,
+                                                    s);
     if (e != cudaSuccess) return fail(PKV_ERR_CUDA, cudaGetErrorString(e));
     note_launches(1);
     return PKV_OK;

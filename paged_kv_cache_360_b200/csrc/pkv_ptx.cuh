@@ -132,6 +132,24 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, uint32_t src
                  : "memory");
 }
 
+// 4-D tiled bulk tensor store shared -> global, otherwise as tma_store_2d.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* tm, uint32_t src, int32_t x,
+                                             int32_t y, int32_t z, int32_t w) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(
+            reinterpret_cast<uint64_t>(tm)),
+        "r"(x), "r"(y), "r"(z), "r"(w), "r"(src)
+        : "memory");
+}
+
+// Close the calling thread's bulk group, then wait until the shared memory
+// its bulk operations read may be reused (their global writes may still be in
+// flight; they are complete when the kernel is).
+__device__ __forceinline__ void bulk_commit_and_wait_read() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // Close the calling thread's bulk group, then wait until every bulk operation
 // it issued has completed (its global writes done).
 __device__ __forceinline__ void bulk_commit_and_wait_all() {
