@@ -317,9 +317,12 @@ __global__ void __launch_bounds__(kCaThreads, 1)
             }
             mma_commit(bar(kCbS + j));
         }
+        // V first: its copies have usually landed while the softmax ran, and a
+        // barrier check between P's arrival and the P V MMAs would sit on the
+        // softmax -> P V path
+        for (int j = 0; j < ntl && ok; ++j) ok = one_wait(bar(kCbV + j), 0, abort_word, a.err);
         for (int j = 0; j < ntl && ok; ++j) {
             if (!(ok = one_wait(bar(kCbP + j), 0, abort_word, a.err))) break;
-            if (!(ok = one_wait(bar(kCbV + j), 0, abort_word, a.err))) break;
             tc_fence_after();
             const uint32_t vs = sb + Lay::kV + j * Lay::kTile;
             // O += P_hi V_j, then O += P_lo V_j (16 tokens = 8 columns of P per step)
