@@ -81,6 +81,28 @@ def test_prefill_chunks_decode_rows_and_empty(dtype, group):
     compare(out, _ref(wl, q, qs), what=f"chunks g={group}")
 
 
+def test_prefill_writes_only_the_query_rows():
+    """Output rows past the last sequence's queries keep what they held, and
+    every written row matches the oracle, for tiles that leave as one bulk
+    store (whole 32-token tiles at g = 4) and ragged last tiles alike."""
+    lens, nq = [300, 64, 129, 37], [96, 64, 33, 37]
+    wl, q, qs = _case(lens, nq, 16, 4, 128, 16, torch.bfloat16, seed=53)
+    extra = 40
+    q_all = torch.cat([q, normal_tensor(np.random.default_rng(54), (extra, 16, 128), torch.bfloat16)])
+    out = torch.full(q_all.shape, float("nan"), dtype=q_all.dtype, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.paged_attention_prefill(
+        out, q_all.cuda(), wl.k_cache.cuda(), wl.v_cache.cuda(),
+        torch.from_numpy(np.ascontiguousarray(wl.block_tables)).cuda(),
+        torch.from_numpy(np.ascontiguousarray(wl.context_lens)).cuda(),
+        torch.from_numpy(qs).cuda(), wl.scale, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    n = int(qs[-1])
+    assert torch.isnan(out[n:].float()).all()
+    compare(out[:n], _ref(wl, q, qs), what="prefill rows of the call")
+
+
 def test_prefill_ignores_garbage_past_the_context():
     lens = [3, 17, 140, 250]
     wl, q, qs = _case(lens, lens, 8, 2, 128, 16, torch.bfloat16, seed=31)
