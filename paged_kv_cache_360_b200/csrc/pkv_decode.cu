@@ -19,9 +19,12 @@
 //     mma.sync m16n8k16, fp32 accumulate, online softmax in base 2);
 //   * the four warps' (m, l, O) are merged in shared memory in warp order.
 //
-// Fixed partitions (partition_size > 0): one CTA per (sequence, kv head,
-// partition of partition_size tokens); a partition's un-normalised O and its
-// (m, l) go to the workspace and reduce_kernel merges partitions p = 0, 1, ...
+// Fixed partitions (partition_size > 0): the balanced schedule below with every
+// segment cut at partition boundaries (partition_size tokens); each partition's
+// un-normalised O and its (m, l) go to a slot of the workspace (a partition
+// split across CTAs is first merged by the chain kernel) and reduce_kernel
+// merges a row's partitions p = 0, 1, ...  A partition_size of at least the
+// table width means no split: decode_kernel, one CTA per (sequence, kv head).
 //
 // Balanced (partition_size == 0): a persistent grid of G CTAs (the resident
 // count).  The work is the list of units (sequence b, kv head hk, logical block)
