@@ -290,13 +290,17 @@ size_t paged_attention_shared_prefix_workspace_bytes(const pkv_cache_desc* desc,
  * probabilities enter P V rounded to `dtype` (for query rows that see at most
  * 128 tokens their rounding residual is added by a second product); output
  * rounded to `dtype`.  scale must be positive.
- *   out, q          device [num_tokens][num_heads][head_dim], 16-byte aligned;
- *                   rows of a sequence are consecutive, sequences in order.
+ *   out, q          device [num_tokens][num_heads][head_dim], 16-byte aligned,
+ *                   not overlapping; rows of a sequence are consecutive,
+ *                   sequences in order.  A full 128-row query tile of out is
+ *                   written by one bulk tensor store, other rows one by one;
+ *                   rows that belong to no sequence are not written.
  *   k_cache, v_cache device pools, 16-byte aligned (read only).
  *   block_tables    device int32 [num_seqs][max_blocks_per_seq]; entries at or
  *                   past ceil(context_len / block_size) are not read.
  *   context_lens    device int32 [num_seqs].
- *   query_start     device int32 [num_seqs + 1], query_start[num_seqs] = num_tokens.
+ *   query_start     device int32 [num_seqs + 1], non-decreasing from 0,
+ *                   query_start[num_seqs] <= num_tokens.
  *   num_heads / num_kv_heads must be a power of two <= 128.
  *   err_flag        device int32 or NULL (PKV_DEVERR_BAD_BLOCK_ID,
  *                   PKV_DEVERR_BAD_CONTEXT_LEN, PKV_DEVERR_BAD_QUERY_COUNT,
