@@ -780,6 +780,12 @@ extern "C" pkv_status paged_attention_prefill(const pkv_cache_desc* desc, void* 
         return fail(PKV_ERR_INVALID_ARG, "paged_attention_prefill: NULL pointer");
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
         return fail(PKV_ERR_INVALID_ARG, "out, q and the pools must be 16-byte aligned");
+    {
+        const uintptr_t ob = reinterpret_cast<uintptr_t>(out), qb = reinterpret_cast<uintptr_t>(q);
+        const uintptr_t bytes = static_cast<uintptr_t>(num_tokens) * num_heads * desc->head_dim * 2u;
+        if (ob < qb + bytes && qb < ob + bytes)
+            return fail(PKV_ERR_INVALID_ARG, "out must not overlap q");
+    }
     if (static_cast<int64_t>(num_tokens) / (kPfRows / g) + num_seqs > INT32_MAX)
         return fail(PKV_ERR_UNSUPPORTED, "too many query tiles");
 

@@ -148,6 +148,7 @@ def test_prefill_rejects_bad_arguments(lib):
     assert _prefill(lib, d, mb=0) == 1
     assert _prefill(lib, d, qs=None) == 1
     assert _prefill(lib, d, out=ctypes.c_void_p(0x10008)) == 1   # misaligned
+    assert _prefill(lib, d, out=ctypes.c_void_p(0x20000), q=ctypes.c_void_p(0x20400)) == 1  # overlap
     assert _prefill(lib, d, T=0) == 0                    # nothing to do
     assert _prefill(lib, d, B=0) == 0
     assert lib.pkv_last_error().decode()
